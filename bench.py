@@ -1,0 +1,372 @@
+"""Benchmark of the fused two-step quantized all-reduce on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--variant fused|fused_nopayload|staged]
+
+One step = one whole quantized all-reduce of the workload (step-1 quantize
+of every rank, reduce-scatter dequant-sum-requant, all-gather dequant) over
+one batch of seeded synthetic partials already resident in HBM.  Default
+workload: P=4 ranks of fp16 [8192 x 8192] partials (LLaMA-3-70B-shaped
+prefill o_proj partial sums), INT8 in both steps, block 128.  The metric is
+GB/s of input consumed (P*N*2 bytes per step); the roofline object reports
+the algorithmic bytes of the kernel against the measured HBM copy bandwidth.
+
+The N > 1 launch (torchrun, one process per GPU) runs an independent replica
+of the whole P-rank problem on every GPU -- the method's ranks are emulated
+inside one GPU, so there is no data-path collective; NCCL carries only the
+barrier and the max-over-ranks of the timings.  ``value`` is the aggregate
+over all GPUs.
+
+``--impl reference`` times the CPU oracle (the plain definition the kernels
+are checked against) on a bounded sample of the same workload, on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import glob
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from bit_quantized_all_block_b200 import synth  # noqa: E402
+
+WORKLOADS = {w.name: w for w in (synth.SMALL_P2, synth.PREFILL_70B_INT8, synth.PREFILL_70B_INT4,
+                                 *synth.BLOCK_SWEEP_8B, synth.DECODE_P4)}
+DEFAULT_WORKLOAD = synth.PREFILL_70B_INT8.name
+METRIC = "quantized all-reduce input GB/s and % of HBM roofline (1×B200)"
+FALLBACK_HBM_GBS = 6650.0
+KERNEL_SOURCES = sorted(glob.glob(os.path.join(ROOT, "bit_quantized_all_block_b200", "csrc", "*.cu*")))
+
+
+def payload_bytes(w) -> int:
+    """Wire bytes of one quantization of n elements: codes + fp32 scale + u8 zero-point."""
+    return w.n * w.bits // 8 + 5 * (w.n // w.block)
+
+
+def algorithmic_bytes(w, variant: str) -> int:
+    e = 2
+    w2 = payload_bytes(w)
+    w1 = w.P * w2
+    if variant == "fused":
+        return w.P * w.n * e + w.n * e + w1 + w2
+    if variant == "fused_nopayload":
+        return w.P * w.n * e + w.n * e
+    if variant == "staged":
+        return w.P * w.n * e + 2 * w1 + 2 * w2 + w.n * e
+    raise ValueError(variant)
+
+
+def source_hash() -> str:
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        h.update(os.path.basename(p).encode())
+        h.update(open(p, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def read_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def read_traffic(workload: str, variant: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel sources; else None."""
+    p = os.path.join(ROOT, "profiles", f"traffic_{variant}_{workload}.txt")
+    try:
+        kv = dict(line.split(":", 1) for line in open(p).read().splitlines() if ":" in line)
+    except OSError:
+        return None
+    if kv.get("kernel_source_hash", "").strip() != source_hash():
+        return None
+    try:
+        return int(kv["dram_bytes_per_launch"].strip())
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """Samples nvidia-smi SM clocks and throttle reasons during the timed region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        time.sleep(0.25)
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.thread.join(timeout=2)
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, f[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def max_over_ranks(v: float, world: int, device="cuda") -> float:
+    """Max of a per-rank timing over all ranks (the job's time is its slowest rank's)."""
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(bytes_per_gpu: int, world: int, ms: float) -> float:
+    """Whole-job GB/s: every GPU processes bytes_per_gpu in the max-over-ranks time ms."""
+    return world * bytes_per_gpu / (ms * 1e-3) / 1e9
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def run_reference(args, w):
+    """The CPU oracle, as it stands, on a bounded row sample per step (rank 0 only)."""
+    world, rank, _ = dist_setup(args)
+    if rank != 0:
+        return
+    import oracle
+    rows = args.ref_rows
+    xs = synth.workload_partials(w, rows=rows)
+    n_in = xs.size * 2
+    for _ in range(args.warmup):
+        oracle.allreduce(list(xs), w.dtype, w.bits, w.block)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.allreduce(list(xs), w.dtype, w.bits, w.block)
+    dt = (time.perf_counter() - t0) / args.steps
+    value = n_in / dt / 1e9
+    sample = f"first {rows} of {w.T} token rows of every rank ({xs.size} input elements per step)"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(dt * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": w.name, "description": w.describe(), "sample": sample},
+        "cpu_baseline": {"value": round(value, 6), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--variant", default="fused", choices=["fused", "fused_nopayload", "staged"])
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--ref-rows", type=int, default=256,
+                    help="token rows per rank in one reference (oracle) step")
+    ap.add_argument("--cpu-rows", type=int, default=0,
+                    help="token rows per rank for the cpu_baseline sample (0 = the whole workload)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    assert args.warmup >= 3 or args.impl == "reference", "at least 3 warm-up steps"
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+
+    import torch
+    import torch.distributed as dist
+
+    import bit_quantized_all_block_b200 as fc
+
+    world, rank, local = dist_setup(args)
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    # ---- inputs: seeded host generation, identical bytes on every rank -------
+    xs_host = synth.workload_partials(w)
+    tdt = torch.float16 if w.dtype == synth.FP16 else torch.bfloat16
+    xs_pinned = [torch.from_numpy(x.view(np.int16)).view(tdt).pin_memory() for x in xs_host]
+    xs = [x.cuda() for x in xs_pinned]
+    y = torch.empty(w.n, dtype=tdt, device="cuda")
+    s1 = [fc.QBuf.empty(w.n, w.bits, w.block) for _ in range(w.P)]
+    s2 = fc.QBuf.empty(w.n, w.bits, w.block)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        if args.variant == "fused":
+            fc.fc_quantized_allreduce(xs, w.bits, w.block, y=y, step1=s1, step2=s2)
+        elif args.variant == "fused_nopayload":
+            fc.fc_quantized_allreduce(xs, w.bits, w.block, y=y)
+        else:
+            for r in range(w.P):
+                fc.fc_quantize(xs[r], w.bits, w.block, out=s1[r])
+            fc.fc_rs_dequant_sum_requant(s1, w.bits, w.block, out=s2)
+            fc.fc_ag_dequant(s2, tdt, y=y)
+
+    launches_per_step = 1 if args.variant.startswith("fused") else w.P + 2
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    # ---- timed region: K steps, events on the launching stream ---------------
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clocks:
+        barrier()
+        torch.cuda.synchronize()
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    ms = ev0.elapsed_time(ev1) / args.steps
+    ms = max_over_ranks(ms, world)
+
+    # ---- end to end through the public API with host buffers -----------------
+    y_host = torch.empty(w.n, dtype=tdt).pin_memory()
+    for _ in range(2):
+        for r in range(w.P):
+            xs[r].copy_(xs_pinned[r], non_blocking=True)
+        step()
+        y_host.copy_(y, non_blocking=True)
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        for r in range(w.P):
+            xs[r].copy_(xs_pinned[r], non_blocking=True)
+        step()
+        y_host.copy_(y, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms_e2e = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, world)
+
+    in_bytes = w.P * w.n * 2
+    value = job_throughput(in_bytes, world, ms)
+    value_e2e = job_throughput(in_bytes, world, ms_e2e)
+    alg = algorithmic_bytes(w, args.variant)
+    peak, peak_kind = read_peak()
+    achieved = alg / (ms * 1e-3) / 1e9
+    traffic = read_traffic(w.name, args.variant)
+
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "data": "synthetic",
+        "config": {"workload": w.name, "description": w.describe(), "variant": args.variant,
+                   "parallelism": f"replicas x{world} (P={w.P} ranks emulated per GPU)",
+                   "l2": f"inputs larger than L2 ({in_bytes / 1e6:.0f} MB read per step), no flush"},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": traffic,
+                     "peak_kind": f"{peak_kind} copy bandwidth",
+                     "algorithmic_bytes_per_launch": alg if args.variant.startswith("fused") else None,
+                     "algorithmic_bytes_per_step": alg},
+        "e2e": {"value": round(value_e2e, 3), "unit": "GB/s", "h2d_bytes_per_step": in_bytes,
+                "d2h_bytes_per_step": w.n * 2},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks.summary(),
+    }
+
+    # ---- result quality and the CPU baseline (rank 0, N = 1 only) -----------
+    if rank == 0:
+        torch.cuda.synchronize()
+        y_np = y.view(torch.int16).cpu().numpy().view(np.uint16)
+        import torch as _t
+        wide = [_t.from_numpy(x.view(np.int16)).view(tdt).to(_t.float32).numpy() for x in xs_host]
+        S = wide[0].copy()
+        for v in wide[1:]:
+            S += v                                      # fp32, rank order 0..P-1
+        yf = _t.from_numpy(y_np.view(np.int16)).view(tdt).to(_t.float32).numpy().astype(np.float64)
+        err = yf - S.astype(np.float64)
+        mse = float(np.mean(err * err))
+        line["quality"] = {"mse_vs_fp32_sum": mse,
+                           "rel_mse": mse / float(np.mean(S.astype(np.float64) ** 2))}
+        if world == 1 and not args.no_cpu_baseline:
+            import oracle
+            rows = args.cpu_rows or w.T
+            sub = [x[: rows * w.H] for x in xs_host]
+            t0 = time.perf_counter()
+            y_ref, _, _ = oracle.allreduce(sub, w.dtype, w.bits, w.block)
+            dt = time.perf_counter() - t0
+            line["cpu_baseline"] = {
+                "value": round(sum(x.size for x in sub) * 2 / dt / 1e9, 5), "unit": "GB/s", "cores": 1,
+                "kind": "oracle",
+                "sample": f"{rows} of {w.T} token rows per rank, {dt:.1f} s, single thread"}
+            line["quality"]["bit_exact_vs_oracle"] = bool(np.array_equal(y_np[: rows * w.H], y_ref))
+        print(json.dumps(line), flush=True)
+
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

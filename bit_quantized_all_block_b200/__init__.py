@@ -1,1 +1,209 @@
-"""B200-native low-bit two-step quantized all-reduce (Flash Communication)."""
+"""B200-native low-bit two-step quantized all-reduce (Flash Communication).
+
+Thin Python binding of the C ABI declared in ``include/fc.h`` (the library is
+``libfc.so`` next to this file, built by ``python -m
+bit_quantized_all_block_b200.build``).  The functions here carry the C names
+and only marshal arguments: torch CUDA tensors supply device pointers, the
+current torch stream is passed as the CUDA stream, and every step of the
+computation runs in the library's sm_100a kernels.  There is no CPU path: if
+the library is missing or a call fails, an exception is raised.
+
+Method: Flash Communication (sciencestack.ai/paper/2412.04964, TL;DR, Fig. 3-5)
+-- per-block asymmetric INT8/INT4 quantization of tensor-parallel partial
+sums, then a reduce-scatter (dequantize every rank's chunk, sum in fp32 in
+rank order, requantize) and an all-gather (dequantize to fp16/bf16).  Here the
+P ranks are P buffers on one GPU.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfc.so")
+HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "fc.h")
+
+FC_OK = 0
+FC_ERR_INVALID_ARG = 1
+FC_ERR_UNSUPPORTED = 2
+FC_ERR_MISALIGNED = 3
+FC_ERR_CUDA = 4
+
+FC_FP16 = 0
+FC_BF16 = 1
+
+
+class fc_qbuf(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("zps", ctypes.c_void_p)]
+
+
+class FCError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        self.cuda_error = _lib().fc_last_cuda_error() if status == FC_ERR_CUDA else 0
+        msg = f"{what}: {fc_status_string(status)}"
+        if self.cuda_error:
+            msg += f" (cudaError {self.cuda_error})"
+        super().__init__(msg)
+
+
+_LIB = None
+
+
+def _lib():
+    """Load libfc.so (once).  Raises if it has not been built."""
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m bit_quantized_all_block_b200.build` (needs nvcc)")
+        L = ctypes.CDLL(LIB_PATH)
+        P, S, I = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
+        QP = ctypes.POINTER(fc_qbuf)
+        L.fc_payload_sizes.argtypes = [S, I, I, ctypes.POINTER(S), ctypes.POINTER(S)]
+        L.fc_quantize.argtypes = [P, I, S, I, I, QP, P]
+        L.fc_rs_dequant_sum_requant.argtypes = [QP, I, S, I, I, QP, P]
+        L.fc_ag_dequant.argtypes = [QP, S, I, I, I, P, P]
+        L.fc_quantized_allreduce.argtypes = [ctypes.POINTER(P), I, I, S, I, I, P, QP, QP, P]
+        for f in ("fc_payload_sizes", "fc_quantize", "fc_rs_dequant_sum_requant", "fc_ag_dequant",
+                  "fc_quantized_allreduce"):
+            getattr(L, f).restype = I
+        L.fc_status_string.argtypes = [I]
+        L.fc_status_string.restype = ctypes.c_char_p
+        L.fc_last_cuda_error.argtypes = []
+        L.fc_last_cuda_error.restype = I
+        _LIB = L
+    return _LIB
+
+
+def library():
+    """The loaded ctypes library (for callers that want the raw C ABI)."""
+    return _lib()
+
+
+def declared_symbols() -> list[str]:
+    """Names of the functions include/fc.h declares."""
+    text = open(HEADER_PATH).read()
+    return sorted(set(re.findall(r"^\s*(?:fc_status|const char\*|int)\s+(fc_\w+)\s*\(", text, re.M)))
+
+
+def fc_status_string(status: int) -> str:
+    return _lib().fc_status_string(int(status)).decode()
+
+
+def _check(status: int, what: str):
+    if status != FC_OK:
+        raise FCError(status, what)
+
+
+def _dtype_code(t) -> int:
+    import torch
+    if t.dtype == torch.float16:
+        return FC_FP16
+    if t.dtype == torch.bfloat16:
+        return FC_BF16
+    raise TypeError(f"expected float16 or bfloat16, got {t.dtype}")
+
+
+def _torch_dtype(code: int):
+    import torch
+    return torch.float16 if code == FC_FP16 else torch.bfloat16
+
+
+def _stream(stream):
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dev_ptr(t, name: str) -> int:
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    return t.data_ptr()
+
+
+def fc_payload_sizes(n: int, bits: int, block: int) -> tuple[int, int]:
+    cb, nb = ctypes.c_size_t(), ctypes.c_size_t()
+    _check(_lib().fc_payload_sizes(n, bits, block, ctypes.byref(cb), ctypes.byref(nb)), "fc_payload_sizes")
+    return cb.value, nb.value
+
+
+class QBuf:
+    """A payload in device memory: packed codes (uint8), fp32 scales, uint8 zero-points."""
+
+    def __init__(self, codes, scales, zps, n: int, bits: int, block: int):
+        self.codes, self.scales, self.zps = codes, scales, zps
+        self.n, self.bits, self.block = n, bits, block
+
+    @classmethod
+    def empty(cls, n: int, bits: int, block: int, device="cuda"):
+        import torch
+        cb, nb = fc_payload_sizes(n, bits, block)
+        return cls(torch.empty(cb, dtype=torch.uint8, device=device),
+                   torch.empty(nb, dtype=torch.float32, device=device),
+                   torch.empty(nb, dtype=torch.uint8, device=device), n, bits, block)
+
+    def struct(self) -> fc_qbuf:
+        return fc_qbuf(_dev_ptr(self.codes, "codes"), _dev_ptr(self.scales, "scales"),
+                       _dev_ptr(self.zps, "zps"))
+
+    def bytes(self) -> int:
+        return self.codes.numel() + 4 * self.scales.numel() + self.zps.numel()
+
+
+def fc_quantize(x, bits: int, block: int, out: QBuf | None = None, stream=None) -> QBuf:
+    """Step 1 on one rank: quantize the fp16/bf16 tensor x (flattened)."""
+    n = x.numel()
+    out = out or QBuf.empty(n, bits, block, x.device)
+    q = out.struct()
+    _check(_lib().fc_quantize(ctypes.c_void_p(_dev_ptr(x, "x")), _dtype_code(x), n, bits, block,
+                              ctypes.byref(q), _stream(stream)), "fc_quantize")
+    return out
+
+
+def fc_rs_dequant_sum_requant(ins, bits: int, block: int, out: QBuf | None = None, stream=None) -> QBuf:
+    """Reduce-scatter step over the P step-1 payloads ``ins``; returns the step-2 payload."""
+    P = len(ins)
+    n = ins[0].n
+    out = out or QBuf.empty(n, bits, block, ins[0].codes.device)
+    arr = (fc_qbuf * P)(*[q.struct() for q in ins])
+    q2 = out.struct()
+    _check(_lib().fc_rs_dequant_sum_requant(arr, P, n, bits, block, ctypes.byref(q2), _stream(stream)),
+           "fc_rs_dequant_sum_requant")
+    return out
+
+
+def fc_ag_dequant(q: QBuf, out_dtype, y=None, stream=None):
+    """All-gather step: dequantize the step-2 payload to fp16/bf16 (``out_dtype`` a torch dtype)."""
+    import torch
+    code = FC_FP16 if out_dtype == torch.float16 else FC_BF16 if out_dtype == torch.bfloat16 else None
+    if code is None:
+        raise TypeError(f"out_dtype must be float16 or bfloat16, got {out_dtype}")
+    y = torch.empty(q.n, dtype=out_dtype, device=q.codes.device) if y is None else y
+    qs = q.struct()
+    _check(_lib().fc_ag_dequant(ctypes.byref(qs), q.n, q.bits, q.block, code,
+                                ctypes.c_void_p(_dev_ptr(y, "y")), _stream(stream)), "fc_ag_dequant")
+    return y
+
+
+def fc_quantized_allreduce(xs, bits: int, block: int, y=None, step1=None, step2: QBuf | None = None,
+                           stream=None):
+    """Fused two-step quantized all-reduce of the P partials ``xs`` (same shape and dtype).
+
+    ``step1`` (a list of P QBufs) and ``step2`` optionally receive the wire payloads."""
+    import torch
+    P = len(xs)
+    n = xs[0].numel()
+    dt = _dtype_code(xs[0])
+    for x in xs:
+        if x.numel() != n or _dtype_code(x) != dt:
+            raise ValueError("all partials must have the same size and dtype")
+    y = torch.empty(n, dtype=xs[0].dtype, device=xs[0].device) if y is None else y
+    xp = (ctypes.c_void_p * P)(*[_dev_ptr(x, "x") for x in xs])
+    s1 = (fc_qbuf * P)(*[q.struct() for q in step1]) if step1 is not None else None
+    s2 = step2.struct() if step2 is not None else None
+    _check(_lib().fc_quantized_allreduce(xp, P, dt, n, bits, block, ctypes.c_void_p(_dev_ptr(y, "y")),
+                                         s1, ctypes.byref(s2) if s2 is not None else None,
+                                         _stream(stream)), "fc_quantized_allreduce")
+    return y

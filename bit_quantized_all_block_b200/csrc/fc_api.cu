@@ -1,0 +1,310 @@
+// fc_api.cu -- the C ABI (include/fc.h): host-side validation and dispatch.
+//
+// Every entry point validates its arguments completely before it touches the
+// GPU, then launches exactly one kernel on the caller's stream and returns
+// without synchronizing.  Nothing is allocated.
+#include <cuda_runtime.h>
+
+#include <map>
+#include <mutex>
+#include <utility>
+
+#include "../../include/fc.h"
+#include "fc_kernels.cuh"
+
+namespace {
+
+thread_local int g_last_cuda_error = 0;
+
+fc_status cuda_fail(cudaError_t e)
+{
+    g_last_cuda_error = (int)e;
+    return FC_ERR_CUDA;
+}
+
+bool valid_bits(int bits) { return bits == 4 || bits == 8; }
+
+bool valid_block(int block)
+{
+    return block >= 32 && block <= 4096 && (block & (block - 1)) == 0;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Byte ranges [p, p+len) for the overlap checks.
+struct Range {
+    const void* p;
+    size_t len;
+};
+
+bool overlap(Range a, Range b)
+{
+    if (a.len == 0 || b.len == 0)
+        return false;
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(a.p), b0 = reinterpret_cast<uintptr_t>(b.p);
+    return a0 < b0 + b.len && b0 < a0 + a.len;
+}
+
+// Checks a payload's pointers; appends its three ranges to `out`.
+fc_status check_qbuf(const fc_qbuf* q, size_t n, int bits, int block, Range* out)
+{
+    if (q == nullptr || q->codes == nullptr || q->scales == nullptr || q->zps == nullptr)
+        return FC_ERR_INVALID_ARG;
+    if (!aligned16(q->codes) || !aligned16(q->scales) || !aligned16(q->zps))
+        return FC_ERR_MISALIGNED;
+    const size_t nb = n / (size_t)block;
+    out[0] = {q->codes, n * (size_t)bits / 8};
+    out[1] = {q->scales, nb * sizeof(float)};
+    out[2] = {q->zps, nb};
+    return FC_OK;
+}
+
+bool any_overlap(const Range* outs, int nout, const Range* ins, int nin)
+{
+    for (int i = 0; i < nout; i++) {
+        for (int j = 0; j < nin; j++)
+            if (overlap(outs[i], ins[j]))
+                return true;
+        for (int j = i + 1; j < nout; j++)
+            if (overlap(outs[i], outs[j]))
+                return true;
+    }
+    return false;
+}
+
+fc::QPtr qptr(const fc_qbuf* q)
+{
+    if (q == nullptr)
+        return fc::QPtr{nullptr, nullptr, nullptr};
+    return fc::QPtr{q->codes, q->scales, q->zps};
+}
+
+using QuantFnT = cudaError_t (*)(const fc::QuantArgs&, cudaStream_t);
+using RsFnT = cudaError_t (*)(const fc::RsArgs&, cudaStream_t);
+using AgFnT = cudaError_t (*)(const fc::AgArgs&, cudaStream_t);
+using FusedFnT = cudaError_t (*)(const fc::FusedArgs&, cudaStream_t);
+
+// [dtype][bits == 4]
+const QuantFnT kQuant[2][2] = {
+    {fc::launch_quantize<__half, 8>, fc::launch_quantize<__half, 4>},
+    {fc::launch_quantize<__nv_bfloat16, 8>, fc::launch_quantize<__nv_bfloat16, 4>},
+};
+const AgFnT kAg[2][2] = {
+    {fc::launch_ag<__half, 8>, fc::launch_ag<__half, 4>},
+    {fc::launch_ag<__nv_bfloat16, 8>, fc::launch_ag<__nv_bfloat16, 4>},
+};
+// [bits == 4][P - 1]
+const RsFnT kRs[2][8] = {
+    {fc::launch_rs<8, 1>, fc::launch_rs<8, 2>, fc::launch_rs<8, 3>, fc::launch_rs<8, 4>,
+     fc::launch_rs<8, 5>, fc::launch_rs<8, 6>, fc::launch_rs<8, 7>, fc::launch_rs<8, 8>},
+    {fc::launch_rs<4, 1>, fc::launch_rs<4, 2>, fc::launch_rs<4, 3>, fc::launch_rs<4, 4>,
+     fc::launch_rs<4, 5>, fc::launch_rs<4, 6>, fc::launch_rs<4, 7>, fc::launch_rs<4, 8>},
+};
+#define FC_FUSED_ROW(T, B)                                                                        \
+    {fc::launch_fused<T, B, 1>, fc::launch_fused<T, B, 2>, fc::launch_fused<T, B, 3>,            \
+     fc::launch_fused<T, B, 4>, fc::launch_fused<T, B, 5>, fc::launch_fused<T, B, 6>,            \
+     fc::launch_fused<T, B, 7>, fc::launch_fused<T, B, 8>}
+// [dtype][bits == 4][P - 1]
+const FusedFnT kFused[2][2][8] = {
+    {FC_FUSED_ROW(__half, 8), FC_FUSED_ROW(__half, 4)},
+    {FC_FUSED_ROW(__nv_bfloat16, 8), FC_FUSED_ROW(__nv_bfloat16, 4)},
+};
+#undef FC_FUSED_ROW
+
+}  // namespace
+
+namespace fc {
+
+cudaError_t persistent_grid(const void* kernel, size_t n, int* grid)
+{
+    static std::mutex mu;
+    static std::map<std::pair<int, const void*>, int> cache;  // (device, kernel) -> CTAs
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return e;
+    int ctas = 0;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        auto it = cache.find({dev, kernel});
+        if (it != cache.end()) {
+            ctas = it->second;
+        } else {
+            int sms = 0, per_sm = 0;
+            e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+            if (e != cudaSuccess)
+                return e;
+            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, FC_THREADS, 0);
+            if (e != cudaSuccess)
+                return e;
+            ctas = sms * (per_sm > 0 ? per_sm : 1);
+            cache[{dev, kernel}] = ctas;
+        }
+    }
+    const size_t tiles = (n + FC_TILE - 1) / FC_TILE;
+    *grid = (int)(tiles < (size_t)ctas ? tiles : (size_t)ctas);
+    return cudaSuccess;
+}
+
+}  // namespace fc
+
+extern "C" {
+
+fc_status fc_payload_sizes(size_t n, int bits, int block, size_t* code_bytes, size_t* n_blocks)
+{
+    if (!valid_bits(bits) || !valid_block(block) || n % (size_t)block != 0 || code_bytes == nullptr ||
+        n_blocks == nullptr)
+        return FC_ERR_INVALID_ARG;
+    *code_bytes = n * (size_t)bits / 8;
+    *n_blocks = n / (size_t)block;
+    return FC_OK;
+}
+
+fc_status fc_quantize(const void* x, fc_dtype dtype, size_t n, int bits, int block, const fc_qbuf* out,
+                      void* stream)
+{
+    if (!valid_bits(bits) || !valid_block(block) || (dtype != FC_FP16 && dtype != FC_BF16) ||
+        n % (size_t)block != 0)
+        return FC_ERR_INVALID_ARG;
+    if (n == 0)
+        return FC_OK;
+    if (x == nullptr)
+        return FC_ERR_INVALID_ARG;
+    if (!aligned16(x))
+        return FC_ERR_MISALIGNED;
+    Range outs[3];
+    fc_status st = check_qbuf(out, n, bits, block, outs);
+    if (st != FC_OK)
+        return st;
+    const Range in{x, n * 2};
+    if (any_overlap(outs, 3, &in, 1))
+        return FC_ERR_INVALID_ARG;
+    fc::QuantArgs a{x, qptr(out), n, block};
+    cudaError_t e = kQuant[dtype][bits == 4](a, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? FC_OK : cuda_fail(e);
+}
+
+fc_status fc_rs_dequant_sum_requant(const fc_qbuf* in, int P, size_t n, int bits, int block,
+                                    const fc_qbuf* out, void* stream)
+{
+    if (!valid_bits(bits) || !valid_block(block) || P < 1 || P > fc::FC_MAX_P ||
+        n % ((size_t)P * (size_t)block) != 0)
+        return FC_ERR_INVALID_ARG;
+    if (n == 0)
+        return FC_OK;
+    if (in == nullptr)
+        return FC_ERR_INVALID_ARG;
+    Range ins[3 * fc::FC_MAX_P], outs[3];
+    for (int r = 0; r < P; r++) {
+        fc_status st = check_qbuf(&in[r], n, bits, block, ins + 3 * r);
+        if (st != FC_OK)
+            return st;
+    }
+    fc_status st = check_qbuf(out, n, bits, block, outs);
+    if (st != FC_OK)
+        return st;
+    if (any_overlap(outs, 3, ins, 3 * P))
+        return FC_ERR_INVALID_ARG;
+    fc::RsArgs a{};
+    for (int r = 0; r < P; r++)
+        a.in[r] = qptr(&in[r]);
+    a.out = qptr(out);
+    a.n = n;
+    a.block = block;
+    cudaError_t e = kRs[bits == 4][P - 1](a, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? FC_OK : cuda_fail(e);
+}
+
+fc_status fc_ag_dequant(const fc_qbuf* in, size_t n, int bits, int block, fc_dtype out_dtype, void* y,
+                        void* stream)
+{
+    if (!valid_bits(bits) || !valid_block(block) || (out_dtype != FC_FP16 && out_dtype != FC_BF16) ||
+        n % (size_t)block != 0)
+        return FC_ERR_INVALID_ARG;
+    if (n == 0)
+        return FC_OK;
+    Range ins[3];
+    fc_status st = check_qbuf(in, n, bits, block, ins);
+    if (st != FC_OK)
+        return st;
+    if (y == nullptr)
+        return FC_ERR_INVALID_ARG;
+    if (!aligned16(y))
+        return FC_ERR_MISALIGNED;
+    const Range out{y, n * 2};
+    if (any_overlap(&out, 1, ins, 3))
+        return FC_ERR_INVALID_ARG;
+    fc::AgArgs a{qptr(in), y, n, block};
+    cudaError_t e = kAg[out_dtype][bits == 4](a, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? FC_OK : cuda_fail(e);
+}
+
+fc_status fc_quantized_allreduce(const void* const* x, int P, fc_dtype dtype, size_t n, int bits, int block,
+                                 void* y, const fc_qbuf* step1, const fc_qbuf* step2, void* stream)
+{
+    if (!valid_bits(bits) || !valid_block(block) || (dtype != FC_FP16 && dtype != FC_BF16) || P < 1 ||
+        P > fc::FC_MAX_P || n % ((size_t)P * (size_t)block) != 0)
+        return FC_ERR_INVALID_ARG;
+    if (n == 0)
+        return FC_OK;
+    if (x == nullptr || y == nullptr)
+        return FC_ERR_INVALID_ARG;
+    Range ins[fc::FC_MAX_P];
+    for (int r = 0; r < P; r++) {
+        if (x[r] == nullptr)
+            return FC_ERR_INVALID_ARG;
+        if (!aligned16(x[r]))
+            return FC_ERR_MISALIGNED;
+        ins[r] = {x[r], n * 2};
+    }
+    if (!aligned16(y))
+        return FC_ERR_MISALIGNED;
+    Range outs[1 + 3 * (fc::FC_MAX_P + 1)];
+    int nout = 0;
+    outs[nout++] = {y, n * 2};
+    if (step1 != nullptr) {
+        for (int r = 0; r < P; r++) {
+            fc_status st = check_qbuf(&step1[r], n, bits, block, outs + nout);
+            if (st != FC_OK)
+                return st;
+            nout += 3;
+        }
+    }
+    if (step2 != nullptr) {
+        fc_status st = check_qbuf(step2, n, bits, block, outs + nout);
+        if (st != FC_OK)
+            return st;
+        nout += 3;
+    }
+    if (any_overlap(outs, nout, ins, P))
+        return FC_ERR_INVALID_ARG;
+    fc::FusedArgs a{};
+    for (int r = 0; r < P; r++) {
+        a.x[r] = x[r];
+        a.step1[r] = step1 ? qptr(&step1[r]) : fc::QPtr{nullptr, nullptr, nullptr};
+    }
+    a.step2 = qptr(step2);
+    a.y = y;
+    a.n = n;
+    a.block = block;
+    a.write_step1 = step1 != nullptr;
+    a.write_step2 = step2 != nullptr;
+    cudaError_t e = kFused[dtype][bits == 4][P - 1](a, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? FC_OK : cuda_fail(e);
+}
+
+const char* fc_status_string(fc_status status)
+{
+    switch (status) {
+    case FC_OK: return "ok";
+    case FC_ERR_INVALID_ARG: return "invalid argument (size, bits, block, P, NULL or overlapping buffer)";
+    case FC_ERR_UNSUPPORTED: return "unsupported combination";
+    case FC_ERR_MISALIGNED: return "device pointer not 16-byte aligned";
+    case FC_ERR_CUDA: return "CUDA error (see fc_last_cuda_error)";
+    }
+    return "unknown status";
+}
+
+int fc_last_cuda_error(void) { return g_last_cuda_error; }
+
+}  // extern "C"

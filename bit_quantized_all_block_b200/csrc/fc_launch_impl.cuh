@@ -1,0 +1,52 @@
+// fc_launch_impl.cuh -- launcher bodies, included by the instantiation units.
+#pragma once
+
+#include "fc_kernels.cuh"
+
+namespace fc {
+
+template <class T, int BITS>
+cudaError_t launch_quantize(const QuantArgs& a, cudaStream_t st)
+{
+    int grid = 0;
+    cudaError_t e = persistent_grid((const void*)k_quantize<T, BITS>, a.n, &grid);
+    if (e != cudaSuccess)
+        return e;
+    k_quantize<T, BITS><<<grid, FC_THREADS, 0, st>>>(a);
+    return cudaGetLastError();
+}
+
+template <int BITS, int P>
+cudaError_t launch_rs(const RsArgs& a, cudaStream_t st)
+{
+    int grid = 0;
+    cudaError_t e = persistent_grid((const void*)k_rs<BITS, P>, a.n, &grid);
+    if (e != cudaSuccess)
+        return e;
+    k_rs<BITS, P><<<grid, FC_THREADS, 0, st>>>(a);
+    return cudaGetLastError();
+}
+
+template <class T, int BITS>
+cudaError_t launch_ag(const AgArgs& a, cudaStream_t st)
+{
+    int grid = 0;
+    cudaError_t e = persistent_grid((const void*)k_ag<T, BITS>, a.n, &grid);
+    if (e != cudaSuccess)
+        return e;
+    k_ag<T, BITS><<<grid, FC_THREADS, 0, st>>>(a);
+    return cudaGetLastError();
+}
+
+template <class T, int BITS, int P>
+cudaError_t launch_fused(const FusedArgs& a, cudaStream_t st)
+{
+    int grid = 0;
+    cudaError_t e = persistent_grid((const void*)k_fused<T, BITS, P>, a.n, &grid);
+    if (e != cudaSuccess)
+        return e;
+    k_fused<T, BITS, P><<<grid, FC_THREADS, 0, st>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace fc

@@ -15,8 +15,8 @@ Recipe (numpy Philox, seed 0 by default):
   2. for rank r = 0..P-1, from its own stream Philox(seed).jumped(r + 1):
      z_r ~ N(0, 1) of shape (T, H) drawn as float32 in row-major order, and
      x_r = z_r * float32(s_c) (float32 product, broadcast over tokens);
-  3. x_r is rounded to fp16 (numpy astype, round-to-nearest-even) or to bf16
-     (torch .to(bfloat16), round-to-nearest-even).
+  3. x_r is rounded to fp16 or bf16 (torch .to(), round-to-nearest-even;
+     identical to numpy's astype(float16) for fp16).
 The function returns the raw 16-bit patterns so that the CPU oracle and the
 GPU receive identical bytes.
 
@@ -25,6 +25,8 @@ library's tests and benchmark; it holds none of the method's arithmetic.
 """
 from __future__ import annotations
 
+import os
+from concurrent.futures import ThreadPoolExecutor
 from dataclasses import dataclass
 
 import numpy as np
@@ -88,10 +90,8 @@ def channel_scales(rng: np.random.Generator, H: int, frac: float, factor: float)
 
 
 def _to_bits(x32: np.ndarray, dtype: int) -> np.ndarray:
-    if dtype == FP16:
-        return x32.astype(np.float16).view(np.uint16)
-    import torch  # bf16 rounding from torch (RNE); host tensors only
-    t = torch.from_numpy(x32).to(torch.bfloat16)
+    import torch  # host tensors only: torch's CPU conversions round to nearest even
+    t = torch.from_numpy(np.ascontiguousarray(x32)).to(torch.float16 if dtype == FP16 else torch.bfloat16)
     return t.view(torch.int16).numpy().view(np.uint16)
 
 
@@ -106,10 +106,15 @@ def partials(P: int, T: int, H: int, dtype: int, outlier_frac: float, outlier_fa
     s32 = channel_scales(rng, H, outlier_frac, outlier_factor).astype(np.float32)
     R = T if rows is None else min(rows, T)
     out = np.empty((P, R * H), dtype=np.uint16)
-    for r in range(P):
+
+    def one_rank(r):
         rng_r = np.random.Generator(np.random.Philox(seed).jumped(r + 1))
         z = rng_r.standard_normal((R, H), dtype=np.float32)
         out[r] = _to_bits(z * s32[None, :], dtype).ravel()
+
+    # ranks draw from independent streams, so they can be generated concurrently
+    with ThreadPoolExecutor(max_workers=min(P, os.cpu_count() or 1)) as ex:
+        list(ex.map(one_rank, range(P)))
     return out
 
 

@@ -1,0 +1,134 @@
+/*
+ * fc.h -- C ABI of the B200 (sm_100a) low-bit two-step quantized all-reduce.
+ *
+ * The method is Flash Communication ("Flash Communication: Reducing Tensor
+ * Parallelization Bottleneck for Fast Large Language Model Inference",
+ * sciencestack.ai/paper/2412.04964): tensor-parallel activation partial sums
+ * are quantized to a few bits per value before they are exchanged, and the
+ * all-reduce runs in two steps, a reduce-scatter followed by an all-gather
+ * (TL;DR; Fig. 3; Fig. 5 right).  Quantization is per block of contiguous
+ * elements along the hidden dimension (Fig. 4).  This library runs all P
+ * ranks of one all-reduce on one GPU: rank r's partial is a buffer in that
+ * GPU's memory, and "sending" a chunk to its owner is reading it.
+ *
+ * Arithmetic (the page gives no formulas; these are the plainest readings).
+ * For a block of B values v_i (fp32; fp16/bf16 inputs are widened exactly),
+ * at b bits with qmax = 2^b - 1, every operation binary32, round to nearest
+ * even, no fused multiply-add:
+ *   mn = min(0, v_i)   mx = max(0, v_i)
+ *   s  = (mx == mn) ? 1 : (mx - mn) / qmax      inv = 1 / s
+ *   z  = clamp(rne(-mn * inv), 0, qmax)          (uint8 zero-point)
+ *   q_i = clamp(rne(v_i * inv) + z, 0, qmax)     (code)
+ *   xhat_i = (q_i - z) * s
+ * Reduce-scatter: chunk c = elements [c*n/P, (c+1)*n/P) is dequantized from
+ * every rank's step-1 payload and summed in fp32 in rank order 0..P-1 (the
+ * sum starts from rank 0's value), then requantized with the same rules
+ * (step-2 payload).  All-gather: the step-2 payload is dequantized and
+ * rounded (nearest even) to fp16/bf16.  Results are bit-identical to the CPU
+ * definition shipped with the tests.
+ *
+ * Payload layout (structure of arrays, one per quantization):
+ *   codes  : n*b/8 bytes.  INT8: one code per byte.  INT4: two codes per
+ *            byte, element 2j in the low nibble, element 2j+1 in the high.
+ *   scales : n/block fp32, scale of block k at index k.
+ *   zps    : n/block uint8, zero-point of block k at index k.
+ * Block k covers elements [k*block, (k+1)*block) of the flat tensor.
+ *
+ * Conventions for every entry point:
+ *   - Pointers named as device pointers must be CUDA device memory (or
+ *     managed memory) of the current device; arrays of pointers and the
+ *     fc_qbuf structs themselves live in host memory and are read before the
+ *     call returns.  The caller owns every buffer; the library allocates
+ *     nothing and keeps no reference after the call.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and the call returns without synchronizing.
+ *   - Arguments are validated on the host before anything is launched.
+ *     bits must be 4 or 8; block a power of two in [32, 4096]; P in [1, 8];
+ *     n a multiple of block (and of P*block where chunks are involved).
+ *     n == 0 is a no-op returning FC_OK (pointers are then not inspected).
+ *     Every device pointer must be non-NULL and 16-byte aligned.
+ *     Output buffers must not overlap input buffers (checked).
+ *   - Inputs must be finite.  For bf16, every block whose range is nonzero
+ *     must have a range in [2^-100, 2^100]; outside that the scale or its
+ *     reciprocal may not be finite and the results are unspecified (the
+ *     kernels still finish and never trap).
+ *   - A CUDA launch failure returns FC_ERR_CUDA; fc_last_cuda_error() then
+ *     gives the cudaError_t value (per calling thread).
+ */
+#ifndef FC_H
+#define FC_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FC_OK = 0,
+    FC_ERR_INVALID_ARG = 1, /* bad size, bits, block, P, NULL or overlapping buffers */
+    FC_ERR_UNSUPPORTED = 2, /* a combination this build does not provide          */
+    FC_ERR_MISALIGNED = 3,  /* a device pointer is not 16-byte aligned             */
+    FC_ERR_CUDA = 4         /* a CUDA call failed; see fc_last_cuda_error()       */
+} fc_status;
+
+typedef enum { FC_FP16 = 0, FC_BF16 = 1 } fc_dtype;
+
+/* One quantized payload (device pointers), layout as described above. */
+typedef struct {
+    uint8_t* codes;
+    float* scales;
+    uint8_t* zps;
+} fc_qbuf;
+
+/* Sizes of one payload for n elements: *code_bytes = n*bits/8 and
+ * *n_blocks = n/block (entries of scales and of zps).  Host only.
+ * Errors: FC_ERR_INVALID_ARG for bad bits/block, n % block != 0, NULL outputs. */
+fc_status fc_payload_sizes(size_t n, int bits, int block, size_t* code_bytes, size_t* n_blocks);
+
+/* Step 1 on one rank (page: TL;DR, low-bit activation quantization; Fig. 4,
+ * per-block granularity): quantize the n fp16/bf16 values at x (device) into
+ * the payload *out (device buffers).  Requires n % block == 0. */
+fc_status fc_quantize(const void* x, fc_dtype dtype, size_t n, int bits, int block,
+                      const fc_qbuf* out, void* stream);
+
+/* Step 2, reduce-scatter (page: two-step All-Reduce; Fig. 5 right, "before
+ * Reduce-Scatter"): in[0..P-1] are the P ranks' step-1 payloads of n elements
+ * each (host array of P structs of device pointers).  For every chunk c, the
+ * owner's work is done: dequantize chunk c from all P payloads, sum in fp32 in
+ * rank order 0..P-1, requantize.  *out receives the step-2 payload of all n
+ * elements (chunk c at its natural offset, so the P owners' outputs form one
+ * payload).  Requires n % (P*block) == 0. */
+fc_status fc_rs_dequant_sum_requant(const fc_qbuf* in, int P, size_t n, int bits, int block,
+                                    const fc_qbuf* out, void* stream);
+
+/* Step 3, all-gather (page: Fig. 5 right, "before All-Gather"): dequantize the
+ * gathered step-2 payload *in (n elements) and round each value to out_dtype
+ * into y (device, n elements).  Requires n % block == 0. */
+fc_status fc_ag_dequant(const fc_qbuf* in, size_t n, int bits, int block, fc_dtype out_dtype,
+                        void* y, void* stream);
+
+/* The fused all-reduce (page: TL;DR, "a fused CUDA kernel implements the
+ * approach"): x is a host array of P device pointers, each to n fp16/bf16
+ * values (rank r's partial).  Writes the all-reduced result, rounded to dtype,
+ * to y (device, n elements) in one kernel, without materialising the wire
+ * payloads.  When step1 is non-NULL it is a host array of P payloads that
+ * receive every rank's step-1 payload; when step2 is non-NULL it receives the
+ * step-2 payload.  Results are bit-identical to fc_quantize x P, then
+ * fc_rs_dequant_sum_requant, then fc_ag_dequant.  Requires n % (P*block) == 0. */
+fc_status fc_quantized_allreduce(const void* const* x, int P, fc_dtype dtype, size_t n, int bits,
+                                 int block, void* y, const fc_qbuf* step1, const fc_qbuf* step2,
+                                 void* stream);
+
+/* Static description of a status code. */
+const char* fc_status_string(fc_status status);
+
+/* cudaError_t of the last call on this thread that returned FC_ERR_CUDA (0 if none). */
+int fc_last_cuda_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FC_H */

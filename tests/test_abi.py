@@ -1,0 +1,105 @@
+"""The C-ABI library loads on the host and exports everything include/fc.h
+declares; host-only entry points and host-side validation behave as
+documented.  No call here reaches a CUDA API: every validation case fails
+before launch (fake, never-dereferenced pointer values are used)."""
+import ctypes
+
+import pytest
+
+import bit_quantized_all_block_b200 as fc
+
+
+def test_library_exports_every_declared_symbol():
+    names = fc.declared_symbols()
+    assert set(names) >= {"fc_payload_sizes", "fc_quantize", "fc_rs_dequant_sum_requant",
+                          "fc_ag_dequant", "fc_quantized_allreduce", "fc_status_string",
+                          "fc_last_cuda_error"}
+    lib = fc.library()
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_payload_sizes():
+    assert fc.fc_payload_sizes(8192 * 8192, 8, 128) == (8192 * 8192, 8192 * 64)
+    assert fc.fc_payload_sizes(4096, 4, 4096) == (2048, 1)
+    assert fc.fc_payload_sizes(0, 4, 32) == (0, 0)
+    for n, bits, block in [(100, 8, 128), (256, 3, 128), (256, 8, 48), (256, 8, 16), (8192, 8, 8192)]:
+        with pytest.raises(fc.FCError) as e:
+            fc.fc_payload_sizes(n, bits, block)
+        assert e.value.status == fc.FC_ERR_INVALID_ARG
+
+
+def test_status_strings():
+    for st in range(5):
+        assert fc.fc_status_string(st)
+    assert fc.library().fc_last_cuda_error() == 0
+
+
+A = 0x10000000   # fake, 16-byte aligned device addresses (never dereferenced)
+
+
+def qb(base):
+    return fc.fc_qbuf(base, base + 0x1000000, base + 0x2000000)
+
+
+def fused(x, P, n, bits=8, block=128, y=A + 0x40000000, step1=None, step2=None, dtype=0):
+    lib = fc.library()
+    xp = (ctypes.c_void_p * len(x))(*x)
+    s1 = (fc.fc_qbuf * P)(*step1) if step1 is not None else None
+    s2 = ctypes.byref(step2) if step2 is not None else None
+    return lib.fc_quantized_allreduce(xp, P, dtype, n, bits, block, ctypes.c_void_p(y), s1, s2, None)
+
+
+XS = [A + r * 0x1000000 for r in range(8)]
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(P=4, n=4096, bits=3), fc.FC_ERR_INVALID_ARG),
+    (dict(P=4, n=4096, block=48), fc.FC_ERR_INVALID_ARG),
+    (dict(P=4, n=4096, block=16), fc.FC_ERR_INVALID_ARG),
+    (dict(P=4, n=4096 * 4, block=8192), fc.FC_ERR_INVALID_ARG),
+    (dict(P=0, n=4096), fc.FC_ERR_INVALID_ARG),
+    (dict(P=9, n=4096 * 9), fc.FC_ERR_INVALID_ARG),
+    (dict(P=3, n=1024), fc.FC_ERR_INVALID_ARG),           # n % (P*block) != 0
+    (dict(P=4, n=4096, dtype=2), fc.FC_ERR_INVALID_ARG),
+    (dict(P=4, n=4096, y=A + 0x40000008), fc.FC_ERR_MISALIGNED),
+    (dict(P=4, n=4096, y=0), fc.FC_ERR_INVALID_ARG),
+    (dict(P=4, n=4096, y=XS[2] + 512), fc.FC_ERR_INVALID_ARG),   # y overlaps x[2]
+    (dict(P=4, n=0, y=0), fc.FC_OK),                              # empty: no-op
+])
+def test_fused_validation(kw, expect):
+    P = kw.pop("P")
+    assert fused(XS[:max(P, 1)] if P <= 8 else XS + XS[:1], P, **kw) == expect
+
+
+def test_fused_validation_pointers():
+    x = list(XS[:4])
+    x[1] = XS[1] + 4
+    assert fused(x, 4, 4096) == fc.FC_ERR_MISALIGNED
+    x[1] = 0
+    assert fused(x, 4, 4096) == fc.FC_ERR_INVALID_ARG
+    # payload outputs: overlapping each other, or misaligned
+    s1 = [qb(A + 0x50000000 + r * 0x4000000) for r in range(4)]
+    s1[3] = qb(A + 0x50000000)
+    assert fused(XS[:4], 4, 4096, step1=s1) == fc.FC_ERR_INVALID_ARG
+    s2 = fc.fc_qbuf(A + 0x70000000, A + 0x70000004, A + 0x71000000)
+    assert fused(XS[:4], 4, 4096, step2=s2) == fc.FC_ERR_MISALIGNED
+    s2 = fc.fc_qbuf(A + 0x70000000, 0, A + 0x71000000)
+    assert fused(XS[:4], 4, 4096, step2=s2) == fc.FC_ERR_INVALID_ARG
+
+
+def test_staged_validation():
+    lib = fc.library()
+    q = qb(A + 0x50000000)
+    assert lib.fc_quantize(ctypes.c_void_p(A), 0, 4096, 5, 128, ctypes.byref(q), None) == fc.FC_ERR_INVALID_ARG
+    assert lib.fc_quantize(ctypes.c_void_p(A + 2), 0, 4096, 8, 128, ctypes.byref(q), None) == fc.FC_ERR_MISALIGNED
+    assert lib.fc_quantize(ctypes.c_void_p(A), 0, 4000, 8, 128, ctypes.byref(q), None) == fc.FC_ERR_INVALID_ARG
+    qo = qb(A)      # codes overlap x
+    assert lib.fc_quantize(ctypes.c_void_p(A), 0, 4096, 8, 128, ctypes.byref(qo), None) == fc.FC_ERR_INVALID_ARG
+    ins = (fc.fc_qbuf * 2)(qb(A), qb(A + 0x4000000))
+    assert lib.fc_rs_dequant_sum_requant(ins, 2, 4096, 8, 128, ctypes.byref(ins[0]), None) == fc.FC_ERR_INVALID_ARG
+    assert lib.fc_rs_dequant_sum_requant(ins, 2, 4096 + 128, 8, 128, ctypes.byref(q), None) == fc.FC_ERR_INVALID_ARG
+    assert lib.fc_rs_dequant_sum_requant(ins, 2, 0, 8, 128, None, None) == fc.FC_OK
+    assert lib.fc_ag_dequant(ctypes.byref(q), 4096, 8, 128, 0, ctypes.c_void_p(A + 0x50000000), None) == fc.FC_ERR_INVALID_ARG
+    assert lib.fc_ag_dequant(ctypes.byref(q), 4096, 8, 128, 0, ctypes.c_void_p(A + 0x7000000a), None) == fc.FC_ERR_MISALIGNED
+    assert lib.fc_ag_dequant(ctypes.byref(q), 4096, 8, 128, 3, ctypes.c_void_p(A), None) == fc.FC_ERR_INVALID_ARG

@@ -1,0 +1,113 @@
+"""GPU parity: the sm_100a kernels, called through the C ABI, are bit-exact
+with the CPU oracle -- codes, scale bit patterns, zero-points and outputs --
+for the fused kernel (with and without payload outputs) and for the staged
+pipeline, over every block size, both bit widths, both dtypes, P = 1..8,
+multi-tile sizes with ragged tails, and the edge cases of the method."""
+import numpy as np
+import pytest
+import torch
+
+import bit_quantized_all_block_b200 as fc
+import oracle
+from bit_quantized_all_block_b200 import synth
+from tests.gpu_util import assert_payload_equal, assert_y_equal, run_fused, run_staged, to_dev, tdtype
+
+pytestmark = pytest.mark.gpu
+
+BLOCKS = [32, 64, 128, 256, 512, 1024, 2048, 4096]
+
+
+def check_all(xs, dtype, bits, block, staged=True):
+    y_ref, p1_ref, p2_ref = oracle.allreduce(list(xs), dtype, bits, block)
+    xd = to_dev(xs, dtype)
+    y, s1, s2 = run_fused(xd, bits, block)
+    assert_y_equal(y, y_ref, "fused y")
+    for r in range(len(xs)):
+        assert_payload_equal(s1[r], p1_ref[r], f"fused step1[{r}]")
+    assert_payload_equal(s2, p2_ref, "fused step2")
+    y_only, _, _ = run_fused(xd, bits, block, with_payloads=False)
+    assert_y_equal(y_only, y_ref, "fused y (no payloads)")
+    if staged:
+        y_st, s1_st, s2_st = run_staged(xd, bits, block)
+        for r in range(len(xs)):
+            assert_payload_equal(s1_st[r], p1_ref[r], f"staged step1[{r}]")
+        assert_payload_equal(s2_st, p2_ref, "staged step2")
+        assert_y_equal(y_st, y_ref, "staged y")
+
+
+@pytest.mark.parametrize("w", [synth.SMALL_P2, synth.DECODE_P4], ids=lambda w: w.name)
+def test_small_workloads_in_full(w):
+    check_all(synth.workload_partials(w), w.dtype, w.bits, w.block)
+
+
+@pytest.mark.parametrize("dtype", [oracle.FP16, oracle.BF16], ids=["fp16", "bf16"])
+@pytest.mark.parametrize("bits", [8, 4])
+@pytest.mark.parametrize("block", BLOCKS)
+@pytest.mark.parametrize("P", [1, 2, 3, 4, 8])
+def test_sweep_ragged(dtype, bits, block, P):
+    # several 4096-element tiles plus a ragged tail (n not a multiple of 4096)
+    m = (3 * 4096) // (P * block) + 3
+    n = P * block * m
+    seed = block * 10 + P + bits + dtype
+    xs = synth.partials(P, n // block, block, dtype, 0.05, 20.0, seed=seed)
+    check_all(xs, dtype, bits, block, staged=(P in (1, 3, 8)))
+
+
+@pytest.mark.parametrize("dtype", [oracle.FP16, oracle.BF16], ids=["fp16", "bf16"])
+@pytest.mark.parametrize("bits", [8, 4])
+def test_zeros_and_sparse(dtype, bits):
+    P, block = 4, 128
+    xs = synth.uniform_partials(P, P * block * 40, dtype, seed=5, zero_frac=0.9)
+    xs[:, : 2 * block * P] = 0            # whole all-zero blocks in every rank
+    xs[1, 5 * block: 6 * block] = 0x8000 if dtype == oracle.FP16 else 0x8000   # negative zeros
+    check_all(xs, dtype, bits, block)
+
+
+@pytest.mark.parametrize("bits", [8, 4])
+def test_fp16_extremes(bits):
+    """Largest finite, subnormal and mixed-sign values; sums that overflow fp16."""
+    P, block, n = 8, 64, 8 * 64 * 9
+    rng = np.random.default_rng(3)
+    vals = np.array([65504.0, -65504.0, 2.0 ** -24, -(2.0 ** -24), 2.0 ** -14, 1.0, -1.0, 0.0],
+                    dtype=np.float32)
+    x = rng.choice(vals, size=(P, n)).astype(np.float16).view(np.uint16)
+    x[:, :block] = np.float16(65504.0).view(np.uint16)           # block summing to inf
+    x[:, block:2 * block] = np.float16(2.0 ** -24).view(np.uint16)   # subnormal-only block
+    check_all(x, oracle.FP16, bits, block)
+
+
+@pytest.mark.parametrize("bits", [8, 4])
+def test_bf16_wide_and_tiny_ranges(bits):
+    """bf16 blocks with ranges from 2^-90 to 2^90 (inside the documented span)."""
+    P, block = 3, 256
+    nb = 24
+    rng = np.random.default_rng(4)
+    z = rng.standard_normal((P, nb, block)).astype(np.float32)
+    mag = (2.0 ** rng.integers(-90, 90, size=(1, nb, 1))).astype(np.float32)
+    x32 = (z * mag).reshape(P, -1)
+    xs = np.stack([torch.from_numpy(r).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+                   for r in x32])
+    check_all(xs, oracle.BF16, bits, block)
+
+
+def test_single_block_and_empty():
+    for P in (1, 4):
+        xs = synth.uniform_partials(P, P * 128, oracle.FP16, seed=P)
+        check_all(xs, oracle.FP16, 8, 128)
+    # n == 0: a no-op that leaves the output untouched
+    e = [torch.empty(0, dtype=torch.float16, device="cuda") for _ in range(2)]
+    y = torch.full((1,), 7.0, dtype=torch.float16, device="cuda")
+    fc.fc_quantized_allreduce(e, 8, 128, y=y[:0])
+    torch.cuda.synchronize()
+    assert y.item() == 7.0
+
+
+def test_staged_and_fused_calls_on_a_side_stream():
+    xs = synth.uniform_partials(2, 2 * 128 * 64, oracle.FP16, seed=8)
+    y_ref, _, _ = oracle.allreduce(list(xs), oracle.FP16, 8, 128)
+    xd = to_dev(xs, oracle.FP16)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        y = fc.fc_quantized_allreduce(xd, 8, 128)
+    s.synchronize()
+    assert_y_equal(y, y_ref, "side stream")
