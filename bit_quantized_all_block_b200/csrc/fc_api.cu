@@ -115,7 +115,7 @@ const FusedFnT kFused[2][2][8] = {
 
 namespace fc {
 
-cudaError_t persistent_grid(const void* kernel, size_t n, int* grid)
+cudaError_t persistent_grid(const void* kernel, int threads, size_t n, size_t tile, int* grid)
 {
     static std::mutex mu;
     static std::map<std::pair<int, const void*>, int> cache;  // (device, kernel) -> CTAs
@@ -134,14 +134,14 @@ cudaError_t persistent_grid(const void* kernel, size_t n, int* grid)
             e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
             if (e != cudaSuccess)
                 return e;
-            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, FC_THREADS, 0);
+            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, 0);
             if (e != cudaSuccess)
                 return e;
             ctas = sms * (per_sm > 0 ? per_sm : 1);
             cache[{dev, kernel}] = ctas;
         }
     }
-    const size_t tiles = (n + FC_TILE - 1) / FC_TILE;
+    const size_t tiles = (n + tile - 1) / tile;
     *grid = (int)(tiles < (size_t)ctas ? tiles : (size_t)ctas);
     return cudaSuccess;
 }

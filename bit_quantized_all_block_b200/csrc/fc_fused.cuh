@@ -1,0 +1,368 @@
+// fc_fused.cuh -- the fused two-step quantized all-reduce kernel (sm_100a).
+//
+// One pass per block index k: load block k of all P ranks, quantize and
+// dequantize each (step 1), sum the dequantized values in rank order (the
+// reduce-scatter), requantize and dequantize the sum (step 2) and store the
+// fp16/bf16 result (the all-gather); the wire payloads are written only when
+// the caller asks for them.  Flash Communication (sciencestack.ai/paper/
+// 2412.04964), TL;DR: "a fused CUDA kernel implements the approach".
+//
+// The kernel moves ~1 GB per call on the 70B-shaped workload and runs close to
+// both the HBM and the instruction-issue ceilings (about a dozen operations per
+// input element), so it is laid out to cut instructions:
+//  * thread t of a CTA owns E contiguous elements of every rank in the tile
+//    (E = 32 for P <= 4, 16 above, to stay in registers); a block of B elements
+//    is L = B/E consecutive threads, so a 128-block needs 4 threads and 2
+//    shuffle rounds.  All loads and stores of a thread use one base pointer
+//    with immediate offsets; codes leave as 128-bit stores.  Loads go through
+//    L1 because the two halves of each 32-byte sector are read by consecutive
+//    instructions of the same thread;
+//  * the P per-rank scale computations of a block are spread over the lanes
+//    of its group (lane r computes rank r) and broadcast with shuffles;
+//  * the upper code clamp binds only when the block maximum's code rounds to
+//    qmax + 1 -- rare -- so it is checked once per block from the maximum and
+//    applied through a warp-uniform branch; the lower clamp never binds
+//    (see quant_shifted in fc_device.cuh);
+//  * each rank's registers are refilled with the next tile's data as soon as
+//    that rank is consumed, so loads stay in flight during the rest of the
+//    tile (software pipelining without extra registers);
+//  * code bytes are formed only when a payload is written.
+#pragma once
+
+#include "fc_kernels.cuh"
+
+namespace fc {
+
+constexpr int FU_THREADS = 256;
+
+#ifndef FC_FUSED_NC_SMALL_P
+#define FC_FUSED_NC_SMALL_P 2
+#endif
+#ifndef FC_FUSED_MIN_CTAS
+#define FC_FUSED_MIN_CTAS 2
+#endif
+
+template <int P>
+struct FuShape {
+    static constexpr int NC = P <= 4 ? FC_FUSED_NC_SMALL_P : 2;   // 16-byte chunks per thread per rank
+    static constexpr int E = NC * FC_CHUNK;                       // elements per thread per rank
+    static constexpr int TILE = FU_THREADS * E;                   // elements per rank per tile
+};
+
+__device__ __forceinline__ uint4 ld_nc(const void* p)
+{
+    uint4 v;
+    asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ float min3(float a, float b, float c)
+{
+    float r;
+    asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+__device__ __forceinline__ float max3(float a, float b, float c)
+{
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+// In-thread {min, -max} of the fp16/bf16 values of NC chunks.
+template <class T, int NC>
+__device__ __forceinline__ uint32_t local_min_negmax(const uint4* c)
+{
+    using P2 = Pair<T>;
+    using T2 = typename P2::T2;
+    T2 m = as_t2<T2>(c[0].x), M = m;
+#pragma unroll
+    for (int i = 0; i < NC; i++) {
+        const uint32_t w[4] = {c[i].x, c[i].y, c[i].z, c[i].w};
+#pragma unroll
+        for (int k = (i == 0 ? 1 : 0); k < 4; k++) {
+            m = __hmin2(m, as_t2<T2>(w[k]));
+            M = __hmax2(M, as_t2<T2>(w[k]));
+        }
+    }
+    const T2 nM = __hneg2(M);
+    return t2_bits(__hmin2(P2::lows(m, nM), P2::highs(m, nM)));
+}
+
+// Whether the largest code of a block, rne(mx*inv) + z, exceeds qmax.
+__device__ __forceinline__ bool top_code_overflows(float mx, const BlockQ& b)
+{
+    const float r = __fadd_rn(__fadd_rn(__fmul_rn(mx, b.inv), FC_MAGIC), b.zf);
+    return r > b.cq;
+}
+
+// Pack the 8 shifted codes of one chunk into the thread's code words:
+// INT8 -> words[2c], words[2c+1]; INT4 -> words[c].
+template <int BITS>
+__device__ __forceinline__ void pack_chunk(const float* sh, uint32_t* words, int c)
+{
+    if constexpr (BITS == 8) {
+        words[2 * c] = pack4_u8(sh);
+        words[2 * c + 1] = pack4_u8(sh + 4);
+    } else {
+        words[c] = pack8_u4(sh);
+    }
+}
+
+// Store a thread's E codes (E*BITS/8 contiguous bytes) at element offset e.
+template <int BITS, int NC>
+__device__ __forceinline__ void store_thread_codes(uint8_t* codes, size_t e, const uint32_t* w)
+{
+    constexpr int NW = NC * BITS / 4;   // 32-bit words: INT8 2 per chunk, INT4 1 per chunk
+    uint8_t* p = codes + e * BITS / 8;
+    if constexpr (NW % 4 == 0) {
+#pragma unroll
+        for (int i = 0; i < NW; i += 4)
+            st_stream(p + 4 * i, make_uint4(w[i], w[i + 1], w[i + 2], w[i + 3]));
+    } else {
+        st_stream(p, make_uint2(w[0], w[1]));
+    }
+}
+
+// Step-1 work on one rank's values, chunk by chunk: quantize, dequantize,
+// accumulate in rank order; optionally store codes, scale and zero-point.
+template <class T, int BITS, int NC, bool CLAMP, bool FIRST>
+__device__ __forceinline__ void rank_body(const uint4* raw, const BlockQ& b, float* acc, bool store,
+                                          const QPtr& out, size_t e, bool leader, size_t k)
+{
+    using P2 = Pair<T>;
+    using T2 = typename P2::T2;
+    const float cqz = __fsub_rn(b.cq, b.zf);   // FC_MAGIC + qmax - z (exact)
+    uint32_t words[NC * BITS / 4];
+#pragma unroll
+    for (int c = 0; c < NC; c++) {
+        const uint32_t w[4] = {raw[c].x, raw[c].y, raw[c].z, raw[c].w};
+        float r[8];
+#pragma unroll
+        for (int h = 0; h < 4; h++) {
+            const float2 v = P2::to_f2(as_t2<T2>(w[h]));
+            r[2 * h] = __fadd_rn(__fmul_rn(v.x, b.inv), FC_MAGIC);       // FC_MAGIC + rne(v*inv)
+            r[2 * h + 1] = __fadd_rn(__fmul_rn(v.y, b.inv), FC_MAGIC);
+        }
+#pragma unroll
+        for (int i = 0; i < 8; i++) {
+            if (CLAMP)
+                r[i] = fminf(r[i], cqz);
+            const float xh = __fmul_rn(__fsub_rn(r[i], FC_MAGIC), b.s);  // (q - z) * s
+            acc[c * 8 + i] = FIRST ? xh : __fadd_rn(acc[c * 8 + i], xh);
+        }
+        if (store) {
+            float sh[8];
+#pragma unroll
+            for (int i = 0; i < 8; i++)
+                sh[i] = __fadd_rn(r[i], b.zf);                            // FC_MAGIC + q
+            pack_chunk<BITS>(sh, words, c);
+        }
+    }
+    if (store) {
+        store_thread_codes<BITS, NC>(out.codes, e, words);
+        if (leader) {
+            out.scales[k] = b.s;
+            out.zps[k] = (uint8_t)b.z;
+        }
+    }
+}
+
+// Step 2 on the sums, chunk by chunk: requantize, dequantize, store y (+ payload).
+template <class T, int BITS, int NC, bool CLAMP>
+__device__ __forceinline__ void sum_body(const float* acc, const BlockQ& b, T* y, bool store,
+                                         const QPtr& out, size_t e, bool leader, size_t k)
+{
+    const float cqz = __fsub_rn(b.cq, b.zf);
+    uint32_t words[NC * BITS / 4];
+#pragma unroll
+    for (int c = 0; c < NC; c++) {
+        float r[8], o[8];
+#pragma unroll
+        for (int i = 0; i < 8; i++) {
+            r[i] = __fadd_rn(__fmul_rn(acc[c * 8 + i], b.inv), FC_MAGIC);
+            if (CLAMP)
+                r[i] = fminf(r[i], cqz);
+            o[i] = __fmul_rn(__fsub_rn(r[i], FC_MAGIC), b.s);
+        }
+        st_stream(y + e + c * FC_CHUNK, narrow8<T>(o));
+        if (store) {
+            float sh[8];
+#pragma unroll
+            for (int i = 0; i < 8; i++)
+                sh[i] = __fadd_rn(r[i], b.zf);
+            pack_chunk<BITS>(sh, words, c);
+        }
+    }
+    if (store) {
+        store_thread_codes<BITS, NC>(out.codes, e, words);
+        if (leader) {
+            out.scales[k] = b.s;
+            out.zps[k] = (uint8_t)b.z;
+        }
+    }
+}
+
+__device__ __forceinline__ BlockQ shfl_blockq(const BlockQ& mine, int src, float cq)
+{
+    BlockQ b;
+    b.s = __shfl_sync(0xffffffffu, mine.s, src);
+    b.inv = __shfl_sync(0xffffffffu, mine.inv, src);
+    b.z = __shfl_sync(0xffffffffu, mine.z, src);
+    b.zf = (float)b.z;
+    b.mz = __uint_as_float(FC_MAGIC_BITS + (uint32_t)b.z);
+    b.cq = cq;
+    return b;
+}
+
+template <class T, int NC>
+__device__ __forceinline__ void load_chunks(uint4* raw, const T* p)
+{
+#pragma unroll
+    for (int c = 0; c < NC; c++)
+        raw[c] = ld_nc(p + c * FC_CHUNK);
+}
+
+template <class T, int BITS, int P>
+__global__ void __launch_bounds__(FU_THREADS, FC_FUSED_MIN_CTAS) k_fused(const FusedArgs a)
+{
+    using P2 = Pair<T>;
+    using T2 = typename P2::T2;
+    constexpr int NC = FuShape<P>::NC, E = FuShape<P>::E, TILE = FuShape<P>::TILE;
+    __shared__ uint32_t red16[P][FU_THREADS / 32];
+    __shared__ float2 red32[FU_THREADS / 32];
+
+    const int L = a.block / E;                 // threads per block (1 .. 256)
+    const int j = threadIdx.x % L;             // member index inside the block
+    const int Lw = L < 32 ? L : 32;            // threads of the block inside this warp
+    const int lane = threadIdx.x & 31;
+    const int grp = lane & ~(Lw - 1);          // first lane of my group in the warp
+    const bool split = Lw >= P;                // lane r of the group computes rank r
+    const size_t toff = (size_t)threadIdx.x * E;
+    const size_t stride = (size_t)gridDim.x * TILE;
+    const float cq = __uint_as_float(FC_MAGIC_BITS + (uint32_t)((1 << BITS) - 1));
+
+    const int lg_block = __ffs(a.block) - 1;   // block is a power of two
+
+    uint4 raw[P][NC];
+    {
+        const size_t e0 = (size_t)blockIdx.x * TILE + toff;
+#pragma unroll
+        for (int r = 0; r < P; r++) {
+            if (e0 < a.n) {
+                load_chunks<T, NC>(raw[r], static_cast<const T*>(a.x[r]) + e0);
+            } else {
+#pragma unroll
+                for (int c = 0; c < NC; c++)
+                    raw[r][c] = make_uint4(0, 0, 0, 0);
+            }
+        }
+    }
+    for (size_t base = (size_t)blockIdx.x * TILE; base < a.n; base += stride) {
+        // My elements [e, e + E) lie inside one block; it is valid iff e < n
+        // (blocks never straddle n because n is a multiple of the block).
+        const size_t e = base + toff;
+        const bool valid = e < a.n;
+        const bool valid_next = e + stride < a.n;
+        const size_t k = e >> lg_block;
+
+        // ---- block extremes of every rank (packed {min, -max}) -------------
+        uint32_t u[P];
+#pragma unroll
+        for (int r = 0; r < P; r++)
+            u[r] = local_min_negmax<T, NC>(raw[r]);
+        for (int o = 1; o < Lw; o <<= 1) {
+#pragma unroll
+            for (int r = 0; r < P; r++)
+                u[r] = t2_bits(__hmin2(as_t2<T2>(u[r]), as_t2<T2>(__shfl_xor_sync(0xffffffffu, u[r], o))));
+        }
+        if (L > 32) {                           // blocks that span warps
+            if (lane == 0) {
+#pragma unroll
+                for (int r = 0; r < P; r++)
+                    red16[r][threadIdx.x >> 5] = u[r];
+            }
+            __syncthreads();
+            const int nw = L >> 5, w0 = (threadIdx.x / L) * nw;
+#pragma unroll
+            for (int r = 0; r < P; r++) {
+                uint32_t v = red16[r][w0];
+                for (int i = 1; i < nw; i++)
+                    v = t2_bits(__hmin2(as_t2<T2>(v), as_t2<T2>(red16[r][w0 + i])));
+                u[r] = v;
+            }
+            __syncthreads();
+        }
+
+        // ---- step-1 scales: one lane per rank when the group is wide enough --
+        BlockQ mine;
+        bool clamp1 = false;
+        if (split) {
+            const int me = lane - grp;
+            uint32_t um = u[0];
+#pragma unroll
+            for (int r = 1; r < P; r++)
+                um = (me == r) ? u[r] : um;
+            const T2 t = as_t2<T2>(um);
+            const float mx = fmaxf(-P2::hi(t), 0.0f);
+            mine = block_q<BITS>(fminf(P2::lo(t), 0.0f), mx);
+            clamp1 = __any_sync(0xffffffffu, top_code_overflows(mx, mine));
+        }
+
+        float acc[E];
+        const bool leader = valid && j == 0;
+        const bool store1 = a.write_step1 && valid;
+#pragma unroll
+        for (int r = 0; r < P; r++) {
+            BlockQ b;
+            bool clamp = clamp1;
+            if (split) {
+                b = shfl_blockq(mine, grp + r, cq);
+            } else {
+                const T2 t = as_t2<T2>(u[r]);
+                const float mx = fmaxf(-P2::hi(t), 0.0f);
+                b = block_q<BITS>(fminf(P2::lo(t), 0.0f), mx);
+                clamp = __any_sync(0xffffffffu, top_code_overflows(mx, b));
+            }
+            if (r == 0) {
+                if (clamp)
+                    rank_body<T, BITS, NC, true, true>(raw[r], b, acc, store1, a.step1[r], e, leader, k);
+                else
+                    rank_body<T, BITS, NC, false, true>(raw[r], b, acc, store1, a.step1[r], e, leader, k);
+            } else {
+                if (clamp)
+                    rank_body<T, BITS, NC, true, false>(raw[r], b, acc, store1, a.step1[r], e, leader, k);
+                else
+                    rank_body<T, BITS, NC, false, false>(raw[r], b, acc, store1, a.step1[r], e, leader, k);
+            }
+            if (valid_next)   // refill rank r with the next tile while this one finishes
+                load_chunks<T, NC>(raw[r], static_cast<const T*>(a.x[r]) + e + stride);
+        }
+
+        // ---- step 2: requantize the sum ---------------------------------------
+        float mn = fminf(acc[0], 0.0f), mx = fmaxf(acc[0], 0.0f);
+#pragma unroll
+        for (int i = 1; i + 1 < E; i += 2) {
+            mn = min3(mn, acc[i], acc[i + 1]);
+            mx = max3(mx, acc[i], acc[i + 1]);
+        }
+        mn = fminf(mn, acc[E - 1]);
+        mx = fmaxf(mx, acc[E - 1]);
+        group_minmax_f32(mn, mx, L, red32);
+        const BlockQ b2 = block_q<BITS>(mn, mx);
+        const bool clamp2 = __any_sync(0xffffffffu, top_code_overflows(mx, b2));
+        if (valid) {
+            T* y = static_cast<T*>(a.y);
+            const bool store2 = a.write_step2 != 0;
+            if (clamp2)
+                sum_body<T, BITS, NC, true>(acc, b2, y, store2, a.step2, e, leader, k);
+            else
+                sum_body<T, BITS, NC, false>(acc, b2, y, store2, a.step2, e, leader, k);
+        }
+    }
+}
+
+}  // namespace fc

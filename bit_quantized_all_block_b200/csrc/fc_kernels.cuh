@@ -4,6 +4,7 @@
 // k_rs         reduce-scatter (all chunks)   P step-1 payloads -> step-2 payload
 // k_ag         all-gather dequantization     step-2 payload -> y
 // k_fused      the whole all-reduce          P partials -> y (+ optional payloads)
+//              (fc_fused.cuh)
 //
 // All four are HBM-bandwidth bound elementwise/reduction kernels (no dense
 // contraction, so no tensor cores): persistent CTAs stride over tiles of
@@ -85,7 +86,7 @@ __global__ void __launch_bounds__(FC_THREADS) k_quantize(const QuantArgs a)
             store_codes<BITS>(a.out.codes, e0, sh);
             store_codes<BITS>(a.out.codes, e1, sh + 8);
             if (G.j == 0) {
-                const size_t k = blk0 / a.block;
+                const size_t k = blk0 >> (__ffs(a.block) - 1);
                 a.out.scales[k] = b.s;
                 a.out.zps[k] = (uint8_t)b.z;
             }
@@ -105,7 +106,7 @@ __global__ void __launch_bounds__(FC_THREADS) k_rs(const RsArgs a)
     for (size_t base = (size_t)blockIdx.x * FC_TILE; base < a.n; base += (size_t)gridDim.x * FC_TILE) {
         const size_t blk0 = base + (size_t)G.g * a.block;
         const bool valid = blk0 < a.n;
-        const size_t k = valid ? blk0 / a.block : 0;
+        const size_t k = valid ? blk0 >> (__ffs(a.block) - 1) : 0;
         const size_t e0 = base + (size_t)G.c0 * FC_CHUNK, e1 = base + (size_t)G.c1 * FC_CHUNK;
         uint32_t w[P][2][2];
         float s[P];
@@ -170,7 +171,7 @@ __global__ void __launch_bounds__(FC_THREADS) k_ag(const AgArgs a)
         const size_t blk0 = base + (size_t)G.g * a.block;
         if (blk0 >= a.n)
             continue;
-        const size_t k = blk0 / a.block;
+        const size_t k = blk0 >> (__ffs(a.block) - 1);
         const size_t e0 = base + (size_t)G.c0 * FC_CHUNK, e1 = base + (size_t)G.c1 * FC_CHUNK;
         uint32_t w0[2], w1[2];
         load_codes<BITS>(a.in.codes, e0, w0);
@@ -188,94 +189,14 @@ __global__ void __launch_bounds__(FC_THREADS) k_ag(const AgArgs a)
     }
 }
 
-// ---------------------------------------------------------------------------
-// The fused all-reduce: for every block index, quantize and dequantize the
-// block of every rank (step 1), sum in rank order (RS), requantize and
-// dequantize (step 2) and write the fp16/bf16 result (AG) -- one pass over
-// the inputs, one write of the output.
-template <class T, int BITS, int P>
-__global__ void __launch_bounds__(FC_THREADS) k_fused(const FusedArgs a)
-{
-    __shared__ uint32_t red16[FC_THREADS / 32];
-    __shared__ float2 red32[FC_THREADS / 32];
-    const Geo G = geometry(a.block);
-    for (size_t base = (size_t)blockIdx.x * FC_TILE; base < a.n; base += (size_t)gridDim.x * FC_TILE) {
-        const size_t blk0 = base + (size_t)G.g * a.block;
-        const bool valid = blk0 < a.n;
-        const size_t k = valid ? blk0 / a.block : 0;
-        const size_t e0 = base + (size_t)G.c0 * FC_CHUNK, e1 = base + (size_t)G.c1 * FC_CHUNK;
-        uint4 raw[P][2];
-#pragma unroll
-        for (int r = 0; r < P; r++) {
-            if (valid) {
-                const T* xr = static_cast<const T*>(a.x[r]);
-                raw[r][0] = ld_stream(xr + e0);
-                raw[r][1] = ld_stream(xr + e1);
-            } else {
-                raw[r][0] = raw[r][1] = make_uint4(0, 0, 0, 0);
-            }
-        }
-        float acc[FC_ELEMS];
-#pragma unroll
-        for (int r = 0; r < P; r++) {
-            float mn, mx;
-            chunk_minmax<T>(raw[r][0], raw[r][1], G.L, red16, mn, mx);
-            const BlockQ b = block_q<BITS>(mn, mx);
-            float v[FC_ELEMS], sh[FC_ELEMS];
-            widen16<T>(raw[r][0], raw[r][1], v);
-#pragma unroll
-            for (int i = 0; i < FC_ELEMS; i++) {
-                sh[i] = quant_shifted(v[i], b);
-                const float xh = dequant_shifted(sh[i], b);
-                acc[i] = (r == 0) ? xh : __fadd_rn(acc[i], xh);
-            }
-            if (a.write_step1 && valid) {
-                store_codes<BITS>(a.step1[r].codes, e0, sh);
-                store_codes<BITS>(a.step1[r].codes, e1, sh + 8);
-                if (G.j == 0) {
-                    a.step1[r].scales[k] = b.s;
-                    a.step1[r].zps[k] = (uint8_t)b.z;
-                }
-            }
-        }
-        float mn = 0.0f, mx = 0.0f;
-#pragma unroll
-        for (int i = 0; i < FC_ELEMS; i++) {
-            mn = fminf(mn, acc[i]);
-            mx = fmaxf(mx, acc[i]);
-        }
-        group_minmax_f32(mn, mx, G.L, red32);
-        const BlockQ b = block_q<BITS>(mn, mx);
-        float sh[FC_ELEMS], out[FC_ELEMS];
-#pragma unroll
-        for (int i = 0; i < FC_ELEMS; i++) {
-            sh[i] = quant_shifted(acc[i], b);
-            out[i] = dequant_shifted(sh[i], b);
-        }
-        if (valid) {
-            T* y = static_cast<T*>(a.y);
-            st_stream(y + e0, narrow8<T>(out));
-            st_stream(y + e1, narrow8<T>(out + 8));
-            if (a.write_step2) {
-                store_codes<BITS>(a.step2.codes, e0, sh);
-                store_codes<BITS>(a.step2.codes, e1, sh + 8);
-                if (G.j == 0) {
-                    a.step2.scales[k] = b.s;
-                    a.step2.zps[k] = (uint8_t)b.z;
-                }
-            }
-        }
-    }
-}
-
 // Host-side launchers (one explicit instantiation per template in its .cu).
 template <class T, int BITS> cudaError_t launch_quantize(const QuantArgs& a, cudaStream_t st);
 template <int BITS, int P> cudaError_t launch_rs(const RsArgs& a, cudaStream_t st);
 template <class T, int BITS> cudaError_t launch_ag(const AgArgs& a, cudaStream_t st);
 template <class T, int BITS, int P> cudaError_t launch_fused(const FusedArgs& a, cudaStream_t st);
 
-// Persistent grid: enough CTAs to fill every SM at the kernel's occupancy,
-// never more than there are tiles.
-cudaError_t persistent_grid(const void* kernel, size_t n, int* grid);
+// Persistent grid: enough CTAs of `threads` threads to fill every SM at the
+// kernel's occupancy, never more than there are tiles of `tile` elements.
+cudaError_t persistent_grid(const void* kernel, int threads, size_t n, size_t tile, int* grid);
 
 }  // namespace fc

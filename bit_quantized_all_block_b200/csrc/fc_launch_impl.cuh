@@ -1,7 +1,7 @@
 // fc_launch_impl.cuh -- launcher bodies, included by the instantiation units.
 #pragma once
 
-#include "fc_kernels.cuh"
+#include "fc_fused.cuh"
 
 namespace fc {
 
@@ -9,7 +9,7 @@ template <class T, int BITS>
 cudaError_t launch_quantize(const QuantArgs& a, cudaStream_t st)
 {
     int grid = 0;
-    cudaError_t e = persistent_grid((const void*)k_quantize<T, BITS>, a.n, &grid);
+    cudaError_t e = persistent_grid((const void*)k_quantize<T, BITS>, FC_THREADS, a.n, FC_TILE, &grid);
     if (e != cudaSuccess)
         return e;
     k_quantize<T, BITS><<<grid, FC_THREADS, 0, st>>>(a);
@@ -20,7 +20,7 @@ template <int BITS, int P>
 cudaError_t launch_rs(const RsArgs& a, cudaStream_t st)
 {
     int grid = 0;
-    cudaError_t e = persistent_grid((const void*)k_rs<BITS, P>, a.n, &grid);
+    cudaError_t e = persistent_grid((const void*)k_rs<BITS, P>, FC_THREADS, a.n, FC_TILE, &grid);
     if (e != cudaSuccess)
         return e;
     k_rs<BITS, P><<<grid, FC_THREADS, 0, st>>>(a);
@@ -31,7 +31,7 @@ template <class T, int BITS>
 cudaError_t launch_ag(const AgArgs& a, cudaStream_t st)
 {
     int grid = 0;
-    cudaError_t e = persistent_grid((const void*)k_ag<T, BITS>, a.n, &grid);
+    cudaError_t e = persistent_grid((const void*)k_ag<T, BITS>, FC_THREADS, a.n, FC_TILE, &grid);
     if (e != cudaSuccess)
         return e;
     k_ag<T, BITS><<<grid, FC_THREADS, 0, st>>>(a);
@@ -42,10 +42,10 @@ template <class T, int BITS, int P>
 cudaError_t launch_fused(const FusedArgs& a, cudaStream_t st)
 {
     int grid = 0;
-    cudaError_t e = persistent_grid((const void*)k_fused<T, BITS, P>, a.n, &grid);
+    cudaError_t e = persistent_grid((const void*)k_fused<T, BITS, P>, FU_THREADS, a.n, FuShape<P>::TILE, &grid);
     if (e != cudaSuccess)
         return e;
-    k_fused<T, BITS, P><<<grid, FC_THREADS, 0, st>>>(a);
+    k_fused<T, BITS, P><<<grid, FU_THREADS, 0, st>>>(a);
     return cudaGetLastError();
 }
 
