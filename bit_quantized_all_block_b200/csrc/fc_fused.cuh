@@ -95,8 +95,7 @@ __device__ __forceinline__ uint32_t local_min_negmax(const uint4* c)
 // Whether the largest code of a block, rne(mx*inv) + z, exceeds qmax.
 __device__ __forceinline__ bool top_code_overflows(float mx, const BlockQ& b)
 {
-    const float r = __fadd_rn(__fadd_rn(__fmul_rn(mx, b.inv), FC_MAGIC), b.zf);
-    return r > b.cq;
+    return __fadd_rn(round_product_shifted(mx, b.inv), b.zf) > b.cq;
 }
 
 // Pack the 8 shifted codes of one chunk into the thread's code words:
@@ -144,8 +143,8 @@ __device__ __forceinline__ void rank_body(const uint4* raw, const BlockQ& b, flo
 #pragma unroll
         for (int h = 0; h < 4; h++) {
             const float2 v = P2::to_f2(as_t2<T2>(w[h]));
-            r[2 * h] = __fadd_rn(__fmul_rn(v.x, b.inv), FC_MAGIC);       // FC_MAGIC + rne(v*inv)
-            r[2 * h + 1] = __fadd_rn(__fmul_rn(v.y, b.inv), FC_MAGIC);
+            r[2 * h] = round_product_shifted(v.x, b.inv);       // FC_MAGIC + rne(v*inv)
+            r[2 * h + 1] = round_product_shifted(v.y, b.inv);
         }
 #pragma unroll
         for (int i = 0; i < 8; i++) {
@@ -166,7 +165,7 @@ __device__ __forceinline__ void rank_body(const uint4* raw, const BlockQ& b, flo
         store_thread_codes<BITS, NC>(out.codes, e, words);
         if (leader) {
             out.scales[k] = b.s;
-            out.zps[k] = (uint8_t)b.z;
+            out.zps[k] = zp_byte(b);
         }
     }
 }
@@ -183,7 +182,7 @@ __device__ __forceinline__ void sum_body(const float* acc, const BlockQ& b, T* y
         float r[8], o[8];
 #pragma unroll
         for (int i = 0; i < 8; i++) {
-            r[i] = __fadd_rn(__fmul_rn(acc[c * 8 + i], b.inv), FC_MAGIC);
+            r[i] = round_product_shifted(acc[c * 8 + i], b.inv);
             if (CLAMP)
                 r[i] = fminf(r[i], cqz);
             o[i] = __fmul_rn(__fsub_rn(r[i], FC_MAGIC), b.s);
@@ -201,7 +200,7 @@ __device__ __forceinline__ void sum_body(const float* acc, const BlockQ& b, T* y
         store_thread_codes<BITS, NC>(out.codes, e, words);
         if (leader) {
             out.scales[k] = b.s;
-            out.zps[k] = (uint8_t)b.z;
+            out.zps[k] = zp_byte(b);
         }
     }
 }
@@ -211,9 +210,8 @@ __device__ __forceinline__ BlockQ shfl_blockq(const BlockQ& mine, int src, float
     BlockQ b;
     b.s = __shfl_sync(0xffffffffu, mine.s, src);
     b.inv = __shfl_sync(0xffffffffu, mine.inv, src);
-    b.z = __shfl_sync(0xffffffffu, mine.z, src);
-    b.zf = (float)b.z;
-    b.mz = __uint_as_float(FC_MAGIC_BITS + (uint32_t)b.z);
+    b.mz = __shfl_sync(0xffffffffu, mine.mz, src);
+    b.zf = __fsub_rn(b.mz, FC_MAGIC);
     b.cq = cq;
     return b;
 }

@@ -88,7 +88,7 @@ __global__ void __launch_bounds__(FC_THREADS) k_quantize(const QuantArgs a)
             if (G.j == 0) {
                 const size_t k = blk0 >> (__ffs(a.block) - 1);
                 a.out.scales[k] = b.s;
-                a.out.zps[k] = (uint8_t)b.z;
+                a.out.zps[k] = zp_byte(b);
             }
         }
     }
@@ -154,7 +154,7 @@ __global__ void __launch_bounds__(FC_THREADS) k_rs(const RsArgs a)
             store_codes<BITS>(a.out.codes, e1, sh + 8);
             if (G.j == 0) {
                 a.out.scales[k] = b.s;
-                a.out.zps[k] = (uint8_t)b.z;
+                a.out.zps[k] = zp_byte(b);
             }
         }
     }

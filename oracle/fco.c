@@ -27,6 +27,8 @@
  *   z  = clamp(rne(-mn * inv), 0, qmax)                  uint8 zero-point
  *   q_i = clamp(rne(v_i * inv) + z, 0, qmax)             code
  *   xhat_i = (q_i - z) * s                               dequantized value
+ * where rne rounds the exact product to the nearest integer, ties to even
+ * (one rounding: the product is not first rounded to fp32).
  * INT4 codes are packed two per byte, the even element in the low nibble.
  *
  * Two-step all-reduce over P ranks (rank r holds partial x_r of n elements):
@@ -166,10 +168,13 @@ static uint16_t store_elem(float v, int dtype)
 /* quantization"; Fig. 4 block granularity along hidden).                    */
 /* ------------------------------------------------------------------------ */
 
-static int rne_int(float t)
+/* Nearest integer, ties to even, of the exact product a*b of two fp32 values.
+ * The product of two 24-bit significands has at most 48 bits, so it is exact
+ * in double; nearbyint rounds to nearest, ties to even, in the default mode. */
+static int rne_product(float a, float b)
 {
-    /* nearbyintf rounds to nearest, ties to even, in the default mode. */
-    return (int)nearbyintf(t);
+    double t = (double)a * (double)b;
+    return (int)nearbyint(t);
 }
 
 static int clamp_int(int v, int lo, int hi)
@@ -195,8 +200,7 @@ int fco_block_stats(const float* v, int B, int bits, float* s_out, float* inv_ou
     float inv = 1.0f / s;
     if (!isfinite(d) || !isfinite(inv) || s == 0.0f)
         return FCO_ERR_RANGE;
-    float t = (-mn) * inv;
-    int z = clamp_int(rne_int(t), 0, qmax);
+    int z = clamp_int(rne_product(-mn, inv), 0, qmax);
     *s_out = s;
     *inv_out = inv;
     *z_out = z;
@@ -204,12 +208,12 @@ int fco_block_stats(const float* v, int B, int bits, float* s_out, float* inv_ou
 }
 
 /* Code of one value given its block's reciprocal scale and zero-point: round
- * first, then add the zero-point as an integer, then clamp. */
+ * the exact product v*inv first, then add the zero-point as an integer, then
+ * clamp. */
 int fco_quantize_value(float v, float inv, int z, int bits)
 {
     const int qmax = (1 << bits) - 1;
-    float t = v * inv;
-    return clamp_int(rne_int(t) + z, 0, qmax);
+    return clamp_int(rne_product(v, inv) + z, 0, qmax);
 }
 
 /* Dequantized value: one fp32 product of the exact integer (q - z) and s. */

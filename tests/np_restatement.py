@@ -18,8 +18,10 @@ def quantize(v32, bits, B):
     with np.errstate(divide="ignore"):
         s = np.where(d == 0, F32(1), d / F32(qmax)).astype(F32)
         inv = (F32(1) / s).astype(F32)
-    z = np.clip(np.rint((-mn) * inv), 0, qmax).astype(np.int64)
-    q = np.clip(np.rint(v * inv[:, None]).astype(np.int64) + z[:, None], 0, qmax)
+    # integer rounding of the exact product (exact in float64: 24 x 24 bits)
+    f64 = np.float64
+    z = np.clip(np.rint((-mn).astype(f64) * inv.astype(f64)), 0, qmax).astype(np.int64)
+    q = np.clip(np.rint(v.astype(f64) * inv.astype(f64)[:, None]).astype(np.int64) + z[:, None], 0, qmax)
     return q.ravel(), s, z
 
 

@@ -20,11 +20,12 @@ SRC = os.path.join(os.path.dirname(oracle.__file__), "fco.c")
 
 MUTANTS = {
     "range_without_zero": ("float mn = 0.0f, mx = 0.0f;", "float mn = v[0], mx = v[0];"),
-    "zero_point_sign": ("float t = (-mn) * inv;", "float t = mn * inv;"),
-    "zero_point_before_rounding": ("return clamp_int(rne_int(t) + z, 0, qmax);",
-                                   "return clamp_int(rne_int(t + (float)z), 0, qmax);"),
-    "no_code_clamp": ("return clamp_int(rne_int(t) + z, 0, qmax);", "return rne_int(t) + z;"),
-    "ties_away_from_zero": ("return (int)nearbyintf(t);", "return (int)roundf(t);"),
+    "zero_point_sign": ("rne_product(-mn, inv)", "rne_product(mn, inv)"),
+    "zero_point_before_rounding": ("return clamp_int(rne_product(v, inv) + z, 0, qmax);",
+                                   "return clamp_int((int)nearbyint((double)v * inv + z), 0, qmax);"),
+    "no_code_clamp": ("return clamp_int(rne_product(v, inv) + z, 0, qmax);",
+                      "return rne_product(v, inv) + z;"),
+    "ties_away_from_zero": ("return (int)nearbyint(t);", "return (int)round(t);"),
     "high_nibble_first": ("} else if (i % 2 == 0) {", "} else if (i % 2 == 1) {",
                           "return (i % 2 == 0) ? (codes[i / 2] & 0x0f) : (codes[i / 2] >> 4);",
                           "return (i % 2 == 1) ? (codes[i / 2] & 0x0f) : (codes[i / 2] >> 4);"),
