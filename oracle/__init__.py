@@ -105,9 +105,10 @@ def _bind(L):
     L.fco_rs_dequant_sum_requant.argtypes = [P, P, P, I, S, I, I, P, P, P]
     L.fco_ag_dequant.argtypes = [P, P, P, S, I, I, I, P]
     L.fco_allreduce.argtypes = [P, I, I, S, I, I, P, P, P, P, P, P, P]
+    L.fco_allreduce_ex.argtypes = [P, I, I, S, I, I, I, P, P, P, P, P, P, P]
     for name in ("fco_block_stats", "fco_quantize_value", "fco_quantize", "fco_quantize_f32",
                  "fco_dequantize",
-                 "fco_rs_dequant_sum_requant", "fco_ag_dequant", "fco_allreduce"):
+                 "fco_rs_dequant_sum_requant", "fco_ag_dequant", "fco_allreduce", "fco_allreduce_ex"):
         getattr(L, name).restype = I
     return L
 
@@ -250,3 +251,22 @@ def allreduce(xs, dtype: int, bits: int, block: int):
                                _ptr_array([p.zps for p in p1]),
                                _ptr(p2.codes), _ptr(p2.scales), _ptr(p2.zps), _ptr(y)), "allreduce")
     return y, p1, p2
+
+
+def allreduce_ex(xs, dtype: int, bits_rs: int, bits_ag: int, block: int):
+    """Two-step all-reduce with per-step precision (4, 8 or 16 = unquantized).
+
+    Returns (y, step1 payloads or None, step2 payload or None)."""
+    xs = [np.ascontiguousarray(x, dtype=np.uint16).ravel() for x in xs]
+    P, n = len(xs), xs[0].size
+    b1 = bits_rs if bits_rs != 16 else 8
+    b2 = bits_ag if bits_ag != 16 else 8
+    p1 = [Payload(n, b1, block) for _ in range(P)]
+    p2 = Payload(n, b2, block)
+    y = np.zeros(n, dtype=np.uint16)
+    _check(lib().fco_allreduce_ex(_ptr_array(xs), P, dtype, n, bits_rs, bits_ag, block,
+                                  _ptr_array([p.codes for p in p1]), _ptr_array([p.scales for p in p1]),
+                                  _ptr_array([p.zps for p in p1]),
+                                  _ptr(p2.codes), _ptr(p2.scales), _ptr(p2.zps), _ptr(y)), "allreduce_ex")
+    return y, (p1 if bits_rs != 16 else None), (p2 if bits_ag != 16 else None)
+

@@ -393,3 +393,73 @@ int fco_allreduce(const uint16_t* const* x, int P, int dtype, size_t n, int bits
         return st;
     return fco_ag_dequant(codes2, scales2, zps2, n, bits, block, dtype, y);
 }
+
+/* ------------------------------------------------------------------------ */
+/* Per-step precision (page: Fig. 5 right, "MSE of quantization before       */
+/* Reduce-Scatter (RS) vs. All-Gather (AG)").  bits_rs and bits_ag are each  */
+/* 4, 8 or 16; 16 means that step sends the 16-bit values unquantized:        */
+/*   bits_rs == 16: the RS sums the exactly widened inputs x_r;              */
+/*   bits_ag == 16: the AG sends the fp32 sum rounded to fp16/bf16, so the    */
+/*                  output is that rounding.                                 */
+/* With bits_rs == bits_ag == b this is fco_allreduce.  Payload outputs of a  */
+/* step that is not quantized are not written (they may be NULL).            */
+/* ------------------------------------------------------------------------ */
+int fco_allreduce_ex(const uint16_t* const* x, int P, int dtype, size_t n, int bits_rs, int bits_ag,
+                     int block, uint8_t* const* codes1, float* const* scales1, uint8_t* const* zps1,
+                     uint8_t* codes2, float* scales2, uint8_t* zps2, uint16_t* y)
+{
+    int bq = bits_rs != 16 ? bits_rs : (bits_ag != 16 ? bits_ag : 8);
+    int st = check_shape(n, bq, block);
+    if (st != FCO_OK || P < 1 || n % ((size_t)P * (size_t)block) != 0 ||
+        (bits_rs != 4 && bits_rs != 8 && bits_rs != 16) || (bits_ag != 4 && bits_ag != 8 && bits_ag != 16) ||
+        (dtype != FCO_FP16 && dtype != FCO_BF16))
+        return FCO_ERR_ARG;
+    /* step 1: every rank's contribution as the RS receives it */
+    float* contrib = (float*)malloc(sizeof(float) * n * (size_t)P);
+    float* acc = (float*)malloc(sizeof(float) * (size_t)block);
+    if (!contrib || !acc) {
+        free(contrib);
+        free(acc);
+        return FCO_ERR_ARG;
+    }
+    for (int r = 0; r < P && st == FCO_OK; r++) {
+        float* c = contrib + (size_t)r * n;
+        if (bits_rs == 16) {
+            for (size_t i = 0; i < n; i++)
+                c[i] = load_elem(x[r], i, dtype);
+        } else {
+            st = fco_quantize(x[r], dtype, n, bits_rs, block, codes1[r], scales1[r], zps1[r]);
+            if (st == FCO_OK)
+                st = fco_dequantize(codes1[r], scales1[r], zps1[r], n, bits_rs, block, c);
+        }
+    }
+    /* RS per owned chunk, then AG of every chunk */
+    const size_t chunk = n / (size_t)P;
+    for (int cidx = 0; cidx < P && st == FCO_OK; cidx++) {
+        for (size_t b0 = (size_t)cidx * chunk; b0 < (size_t)(cidx + 1) * chunk && st == FCO_OK;
+             b0 += (size_t)block) {
+            size_t k = b0 / (size_t)block;
+            for (int i = 0; i < block; i++) {
+                float a = contrib[b0 + (size_t)i];
+                for (int r = 1; r < P; r++)
+                    a = a + contrib[(size_t)r * n + b0 + (size_t)i];
+                acc[i] = a;
+            }
+            if (bits_ag == 16) {
+                for (int i = 0; i < block; i++)
+                    y[b0 + (size_t)i] = store_elem(acc[i], dtype);
+            } else {
+                st = quantize_block(acc, block, bits_ag, k, codes2, scales2, zps2);
+                for (int i = 0; i < block && st == FCO_OK; i++) {
+                    size_t e = b0 + (size_t)i;
+                    float v = fco_dequantize_value(get_code(codes2, e, bits_ag), scales2[k], zps2[k]);
+                    y[e] = store_elem(v, dtype);
+                }
+            }
+        }
+    }
+    free(contrib);
+    free(acc);
+    return st;
+}
+
