@@ -66,8 +66,9 @@ def _lib():
         L.fc_rs_dequant_sum_requant.argtypes = [QP, I, S, I, I, QP, P]
         L.fc_ag_dequant.argtypes = [QP, S, I, I, I, P, P]
         L.fc_quantized_allreduce.argtypes = [ctypes.POINTER(P), I, I, S, I, I, P, QP, QP, P]
+        L.fc_quantized_allreduce_ex.argtypes = [ctypes.POINTER(P), I, I, S, I, I, I, P, QP, QP, P]
         for f in ("fc_payload_sizes", "fc_quantize", "fc_rs_dequant_sum_requant", "fc_ag_dequant",
-                  "fc_quantized_allreduce"):
+                  "fc_quantized_allreduce", "fc_quantized_allreduce_ex"):
             getattr(L, f).restype = I
         L.fc_status_string.argtypes = [I]
         L.fc_status_string.restype = ctypes.c_char_p
@@ -207,3 +208,25 @@ def fc_quantized_allreduce(xs, bits: int, block: int, y=None, step1=None, step2:
                                          s1, ctypes.byref(s2) if s2 is not None else None,
                                          _stream(stream)), "fc_quantized_allreduce")
     return y
+
+
+def fc_quantized_allreduce_ex(xs, bits_rs: int, bits_ag: int, block: int, y=None, step1=None,
+                              step2: QBuf | None = None, stream=None):
+    """Fused all-reduce with a width per step (4, 8 or 16 = unquantized step)."""
+    import torch
+    P = len(xs)
+    n = xs[0].numel()
+    dt = _dtype_code(xs[0])
+    for x in xs:
+        if x.numel() != n or _dtype_code(x) != dt:
+            raise ValueError("all partials must have the same size and dtype")
+    y = torch.empty(n, dtype=xs[0].dtype, device=xs[0].device) if y is None else y
+    xp = (ctypes.c_void_p * P)(*[_dev_ptr(x, "x") for x in xs])
+    s1 = (fc_qbuf * P)(*[q.struct() for q in step1]) if step1 is not None else None
+    s2 = step2.struct() if step2 is not None else None
+    _check(_lib().fc_quantized_allreduce_ex(xp, P, dt, n, bits_rs, bits_ag, block,
+                                            ctypes.c_void_p(_dev_ptr(y, "y")), s1,
+                                            ctypes.byref(s2) if s2 is not None else None,
+                                            _stream(stream)), "fc_quantized_allreduce_ex")
+    return y
+

@@ -100,16 +100,26 @@ const RsFnT kRs[2][8] = {
     {fc::launch_rs<4, 1>, fc::launch_rs<4, 2>, fc::launch_rs<4, 3>, fc::launch_rs<4, 4>,
      fc::launch_rs<4, 5>, fc::launch_rs<4, 6>, fc::launch_rs<4, 7>, fc::launch_rs<4, 8>},
 };
-#define FC_FUSED_ROW(T, B)                                                                        \
-    {fc::launch_fused<T, B, 1>, fc::launch_fused<T, B, 2>, fc::launch_fused<T, B, 3>,            \
-     fc::launch_fused<T, B, 4>, fc::launch_fused<T, B, 5>, fc::launch_fused<T, B, 6>,            \
-     fc::launch_fused<T, B, 7>, fc::launch_fused<T, B, 8>}
-// [dtype][bits == 4][P - 1]
-const FusedFnT kFused[2][2][8] = {
-    {FC_FUSED_ROW(__half, 8), FC_FUSED_ROW(__half, 4)},
-    {FC_FUSED_ROW(__nv_bfloat16, 8), FC_FUSED_ROW(__nv_bfloat16, 4)},
-};
-#undef FC_FUSED_ROW
+// [dtype][width index of the RS step][width index of the AG step][P - 1];
+// width index: 4 -> 0, 8 -> 1, 16 -> 2.  Equal quantized widths exist for
+// every P; the other combinations for P = 2, 4, 8 (NULL elsewhere).
+#define FC_ALLP(T, B1, B2)                                                                        \
+    {fc::launch_fused<T, B1, B2, 1>, fc::launch_fused<T, B1, B2, 2>, fc::launch_fused<T, B1, B2, 3>, \
+     fc::launch_fused<T, B1, B2, 4>, fc::launch_fused<T, B1, B2, 5>, fc::launch_fused<T, B1, B2, 6>, \
+     fc::launch_fused<T, B1, B2, 7>, fc::launch_fused<T, B1, B2, 8>}
+#define FC_P248(T, B1, B2)                                                                        \
+    {nullptr, fc::launch_fused<T, B1, B2, 2>, nullptr, fc::launch_fused<T, B1, B2, 4>,            \
+     nullptr, nullptr, nullptr, fc::launch_fused<T, B1, B2, 8>}
+#define FC_DTYPE(T)                                                                               \
+    {{FC_ALLP(T, 4, 4), FC_P248(T, 4, 8), FC_P248(T, 4, 16)},                                    \
+     {FC_P248(T, 8, 4), FC_ALLP(T, 8, 8), FC_P248(T, 8, 16)},                                    \
+     {FC_P248(T, 16, 4), FC_P248(T, 16, 8), FC_P248(T, 16, 16)}}
+const FusedFnT kFused[2][3][3][8] = {FC_DTYPE(__half), FC_DTYPE(__nv_bfloat16)};
+#undef FC_DTYPE
+#undef FC_P248
+#undef FC_ALLP
+
+int width_index(int bits) { return bits == 4 ? 0 : bits == 8 ? 1 : bits == 16 ? 2 : -1; }
 
 }  // namespace
 
@@ -239,12 +249,19 @@ fc_status fc_ag_dequant(const fc_qbuf* in, size_t n, int bits, int block, fc_dty
     return e == cudaSuccess ? FC_OK : cuda_fail(e);
 }
 
-fc_status fc_quantized_allreduce(const void* const* x, int P, fc_dtype dtype, size_t n, int bits, int block,
-                                 void* y, const fc_qbuf* step1, const fc_qbuf* step2, void* stream)
+fc_status fc_quantized_allreduce_ex(const void* const* x, int P, fc_dtype dtype, size_t n, int bits_rs,
+                                    int bits_ag, int block, void* y, const fc_qbuf* step1,
+                                    const fc_qbuf* step2, void* stream)
 {
-    if (!valid_bits(bits) || !valid_block(block) || (dtype != FC_FP16 && dtype != FC_BF16) || P < 1 ||
+    const int w1 = width_index(bits_rs), w2 = width_index(bits_ag);
+    if (w1 < 0 || w2 < 0 || !valid_block(block) || (dtype != FC_FP16 && dtype != FC_BF16) || P < 1 ||
         P > fc::FC_MAX_P || n % ((size_t)P * (size_t)block) != 0)
         return FC_ERR_INVALID_ARG;
+    if ((bits_rs == 16 && step1 != nullptr) || (bits_ag == 16 && step2 != nullptr))
+        return FC_ERR_INVALID_ARG;   // an unquantized step has no payload
+    const FusedFnT fn = kFused[dtype][w1][w2][P - 1];
+    if (fn == nullptr)
+        return FC_ERR_UNSUPPORTED;
     if (n == 0)
         return FC_OK;
     if (x == nullptr || y == nullptr)
@@ -264,14 +281,14 @@ fc_status fc_quantized_allreduce(const void* const* x, int P, fc_dtype dtype, si
     outs[nout++] = {y, n * 2};
     if (step1 != nullptr) {
         for (int r = 0; r < P; r++) {
-            fc_status st = check_qbuf(&step1[r], n, bits, block, outs + nout);
+            fc_status st = check_qbuf(&step1[r], n, bits_rs, block, outs + nout);
             if (st != FC_OK)
                 return st;
             nout += 3;
         }
     }
     if (step2 != nullptr) {
-        fc_status st = check_qbuf(step2, n, bits, block, outs + nout);
+        fc_status st = check_qbuf(step2, n, bits_ag, block, outs + nout);
         if (st != FC_OK)
             return st;
         nout += 3;
@@ -289,8 +306,16 @@ fc_status fc_quantized_allreduce(const void* const* x, int P, fc_dtype dtype, si
     a.block = block;
     a.write_step1 = step1 != nullptr;
     a.write_step2 = step2 != nullptr;
-    cudaError_t e = kFused[dtype][bits == 4][P - 1](a, static_cast<cudaStream_t>(stream));
+    cudaError_t e = fn(a, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? FC_OK : cuda_fail(e);
+}
+
+fc_status fc_quantized_allreduce(const void* const* x, int P, fc_dtype dtype, size_t n, int bits, int block,
+                                 void* y, const fc_qbuf* step1, const fc_qbuf* step2, void* stream)
+{
+    if (!valid_bits(bits))
+        return FC_ERR_INVALID_ARG;
+    return fc_quantized_allreduce_ex(x, P, dtype, n, bits, bits, block, y, step1, step2, stream);
 }
 
 const char* fc_status_string(fc_status status)

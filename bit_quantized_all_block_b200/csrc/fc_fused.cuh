@@ -5,7 +5,7 @@
 // reduce-scatter), requantize and dequantize the sum (step 2) and store the
 // fp16/bf16 result (the all-gather); the wire payloads are written only when
 // the caller asks for them.  Flash Communication (sciencestack.ai/paper/
-// 2412.04964), TL;DR: "a fused CUDA kernel implements the approach".
+// 2412.04964), TL;DR: the method is implemented as one fused CUDA kernel.
 //
 // The kernel moves ~1 GB per call on the 70B-shaped workload and runs close to
 // both the HBM and the instruction-issue ceilings (about a dozen operations per
@@ -224,12 +224,36 @@ __device__ __forceinline__ void load_chunks(uint4* raw, const T* p)
         raw[c] = ld_nc(p + c * FC_CHUNK);
 }
 
-template <class T, int BITS, int P>
+// Unquantized step 1 (16-bit values sent as they are): the reduce-scatter sums
+// the exactly widened inputs.
+template <class T, int NC, bool FIRST>
+__device__ __forceinline__ void rank_body_plain(const uint4* raw, float* acc)
+{
+    using P2 = Pair<T>;
+    using T2 = typename P2::T2;
+#pragma unroll
+    for (int c = 0; c < NC; c++) {
+        const uint32_t w[4] = {raw[c].x, raw[c].y, raw[c].z, raw[c].w};
+#pragma unroll
+        for (int h = 0; h < 4; h++) {
+            const float2 v = P2::to_f2(as_t2<T2>(w[h]));
+            const int i = c * 8 + 2 * h;
+            acc[i] = FIRST ? v.x : __fadd_rn(acc[i], v.x);
+            acc[i + 1] = FIRST ? v.y : __fadd_rn(acc[i + 1], v.y);
+        }
+    }
+}
+
+// B1 / B2: bits of the reduce-scatter and of the all-gather step, each 4, 8
+// or 16 (16 = that step sends fp16/bf16 values unquantized; Fig. 5 right of
+// the page compares quantizing before RS with quantizing before AG).
+template <class T, int B1, int B2, int P>
 __global__ void __launch_bounds__(FU_THREADS, FC_FUSED_MIN_CTAS) k_fused(const FusedArgs a)
 {
     using P2 = Pair<T>;
     using T2 = typename P2::T2;
     constexpr int NC = FuShape<P>::NC, E = FuShape<P>::E, TILE = FuShape<P>::TILE;
+    constexpr int QB1 = B1 == 16 ? 8 : B1;     // (unused when B1 == 16)
     __shared__ uint32_t red16[P][FU_THREADS / 32];
     __shared__ float2 red32[FU_THREADS / 32];
 
@@ -241,7 +265,7 @@ __global__ void __launch_bounds__(FU_THREADS, FC_FUSED_MIN_CTAS) k_fused(const F
     const bool split = Lw >= P;                // lane r of the group computes rank r
     const size_t toff = (size_t)threadIdx.x * E;
     const size_t stride = (size_t)gridDim.x * TILE;
-    const float cq = __uint_as_float(FC_MAGIC_BITS + (uint32_t)((1 << BITS) - 1));
+    const float cq1 = __uint_as_float(FC_MAGIC_BITS + (uint32_t)((1 << QB1) - 1));
 
     const int lg_block = __ffs(a.block) - 1;   // block is a power of two
 
@@ -266,99 +290,120 @@ __global__ void __launch_bounds__(FU_THREADS, FC_FUSED_MIN_CTAS) k_fused(const F
         const bool valid = e < a.n;
         const bool valid_next = e + stride < a.n;
         const size_t k = e >> lg_block;
+        const bool leader = valid && j == 0;
+        float acc[E];
 
-        // ---- block extremes of every rank (packed {min, -max}) -------------
-        uint32_t u[P];
-#pragma unroll
-        for (int r = 0; r < P; r++)
-            u[r] = local_min_negmax<T, NC>(raw[r]);
-        for (int o = 1; o < Lw; o <<= 1) {
-#pragma unroll
-            for (int r = 0; r < P; r++)
-                u[r] = t2_bits(__hmin2(as_t2<T2>(u[r]), as_t2<T2>(__shfl_xor_sync(0xffffffffu, u[r], o))));
-        }
-        if (L > 32) {                           // blocks that span warps
-            if (lane == 0) {
-#pragma unroll
-                for (int r = 0; r < P; r++)
-                    red16[r][threadIdx.x >> 5] = u[r];
-            }
-            __syncthreads();
-            const int nw = L >> 5, w0 = (threadIdx.x / L) * nw;
+        if constexpr (B1 == 16) {
 #pragma unroll
             for (int r = 0; r < P; r++) {
-                uint32_t v = red16[r][w0];
-                for (int i = 1; i < nw; i++)
-                    v = t2_bits(__hmin2(as_t2<T2>(v), as_t2<T2>(red16[r][w0 + i])));
-                u[r] = v;
+                if (r == 0)
+                    rank_body_plain<T, NC, true>(raw[r], acc);
+                else
+                    rank_body_plain<T, NC, false>(raw[r], acc);
+                if (valid_next)
+                    load_chunks<T, NC>(raw[r], static_cast<const T*>(a.x[r]) + e + stride);
             }
-            __syncthreads();
-        }
-
-        // ---- step-1 scales: one lane per rank when the group is wide enough --
-        BlockQ mine;
-        bool clamp1 = false;
-        if (split) {
-            const int me = lane - grp;
-            uint32_t um = u[0];
+        } else {
+            // ---- block extremes of every rank (packed {min, -max}) ---------
+            uint32_t u[P];
 #pragma unroll
-            for (int r = 1; r < P; r++)
-                um = (me == r) ? u[r] : um;
-            const T2 t = as_t2<T2>(um);
-            const float mx = fmaxf(-P2::hi(t), 0.0f);
-            mine = block_q<BITS>(fminf(P2::lo(t), 0.0f), mx);
-            clamp1 = __any_sync(0xffffffffu, top_code_overflows(mx, mine));
-        }
-
-        float acc[E];
-        const bool leader = valid && j == 0;
-        const bool store1 = a.write_step1 && valid;
+            for (int r = 0; r < P; r++)
+                u[r] = local_min_negmax<T, NC>(raw[r]);
+            for (int o = 1; o < Lw; o <<= 1) {
 #pragma unroll
-        for (int r = 0; r < P; r++) {
-            BlockQ b;
-            bool clamp = clamp1;
+                for (int r = 0; r < P; r++)
+                    u[r] = t2_bits(__hmin2(as_t2<T2>(u[r]), as_t2<T2>(__shfl_xor_sync(0xffffffffu, u[r], o))));
+            }
+            if (L > 32) {                       // blocks that span warps
+                if (lane == 0) {
+#pragma unroll
+                    for (int r = 0; r < P; r++)
+                        red16[r][threadIdx.x >> 5] = u[r];
+                }
+                __syncthreads();
+                const int nw = L >> 5, w0 = (threadIdx.x / L) * nw;
+#pragma unroll
+                for (int r = 0; r < P; r++) {
+                    uint32_t v = red16[r][w0];
+                    for (int i = 1; i < nw; i++)
+                        v = t2_bits(__hmin2(as_t2<T2>(v), as_t2<T2>(red16[r][w0 + i])));
+                    u[r] = v;
+                }
+                __syncthreads();
+            }
+
+            // ---- step-1 scales: one lane per rank when the group is wide enough
+            BlockQ mine;
+            bool clamp1 = false;
             if (split) {
-                b = shfl_blockq(mine, grp + r, cq);
-            } else {
-                const T2 t = as_t2<T2>(u[r]);
+                const int me = lane - grp;
+                uint32_t um = u[0];
+#pragma unroll
+                for (int r = 1; r < P; r++)
+                    um = (me == r) ? u[r] : um;
+                const T2 t = as_t2<T2>(um);
                 const float mx = fmaxf(-P2::hi(t), 0.0f);
-                b = block_q<BITS>(fminf(P2::lo(t), 0.0f), mx);
-                clamp = __any_sync(0xffffffffu, top_code_overflows(mx, b));
+                mine = block_q<QB1>(fminf(P2::lo(t), 0.0f), mx);
+                clamp1 = __any_sync(0xffffffffu, top_code_overflows(mx, mine));
             }
-            if (r == 0) {
-                if (clamp)
-                    rank_body<T, BITS, NC, true, true>(raw[r], b, acc, store1, a.step1[r], e, leader, k);
-                else
-                    rank_body<T, BITS, NC, false, true>(raw[r], b, acc, store1, a.step1[r], e, leader, k);
-            } else {
-                if (clamp)
-                    rank_body<T, BITS, NC, true, false>(raw[r], b, acc, store1, a.step1[r], e, leader, k);
-                else
-                    rank_body<T, BITS, NC, false, false>(raw[r], b, acc, store1, a.step1[r], e, leader, k);
+
+            const bool store1 = a.write_step1 && valid;
+#pragma unroll
+            for (int r = 0; r < P; r++) {
+                BlockQ b;
+                bool clamp = clamp1;
+                if (split) {
+                    b = shfl_blockq(mine, grp + r, cq1);
+                } else {
+                    const T2 t = as_t2<T2>(u[r]);
+                    const float mx = fmaxf(-P2::hi(t), 0.0f);
+                    b = block_q<QB1>(fminf(P2::lo(t), 0.0f), mx);
+                    clamp = __any_sync(0xffffffffu, top_code_overflows(mx, b));
+                }
+                if (r == 0) {
+                    if (clamp)
+                        rank_body<T, QB1, NC, true, true>(raw[r], b, acc, store1, a.step1[r], e, leader, k);
+                    else
+                        rank_body<T, QB1, NC, false, true>(raw[r], b, acc, store1, a.step1[r], e, leader, k);
+                } else {
+                    if (clamp)
+                        rank_body<T, QB1, NC, true, false>(raw[r], b, acc, store1, a.step1[r], e, leader, k);
+                    else
+                        rank_body<T, QB1, NC, false, false>(raw[r], b, acc, store1, a.step1[r], e, leader, k);
+                }
+                if (valid_next)   // refill rank r with the next tile while this one finishes
+                    load_chunks<T, NC>(raw[r], static_cast<const T*>(a.x[r]) + e + stride);
             }
-            if (valid_next)   // refill rank r with the next tile while this one finishes
-                load_chunks<T, NC>(raw[r], static_cast<const T*>(a.x[r]) + e + stride);
         }
 
-        // ---- step 2: requantize the sum ---------------------------------------
-        float mn = fminf(acc[0], 0.0f), mx = fmaxf(acc[0], 0.0f);
+        T* y = static_cast<T*>(a.y);
+        if constexpr (B2 == 16) {
+            // ---- unquantized all-gather: the sum rounded to fp16/bf16 ----------
+            if (valid) {
 #pragma unroll
-        for (int i = 1; i + 1 < E; i += 2) {
-            mn = min3(mn, acc[i], acc[i + 1]);
-            mx = max3(mx, acc[i], acc[i + 1]);
-        }
-        mn = fminf(mn, acc[E - 1]);
-        mx = fmaxf(mx, acc[E - 1]);
-        group_minmax_f32(mn, mx, L, red32);
-        const BlockQ b2 = block_q<BITS>(mn, mx);
-        const bool clamp2 = __any_sync(0xffffffffu, top_code_overflows(mx, b2));
-        if (valid) {
-            T* y = static_cast<T*>(a.y);
-            const bool store2 = a.write_step2 != 0;
-            if (clamp2)
-                sum_body<T, BITS, NC, true>(acc, b2, y, store2, a.step2, e, leader, k);
-            else
-                sum_body<T, BITS, NC, false>(acc, b2, y, store2, a.step2, e, leader, k);
+                for (int c = 0; c < NC; c++)
+                    st_stream(y + e + c * FC_CHUNK, narrow8<T>(acc + c * FC_CHUNK));
+            }
+        } else {
+            // ---- step 2: requantize the sum -------------------------------------
+            float mn = fminf(acc[0], 0.0f), mx = fmaxf(acc[0], 0.0f);
+#pragma unroll
+            for (int i = 1; i + 1 < E; i += 2) {
+                mn = min3(mn, acc[i], acc[i + 1]);
+                mx = max3(mx, acc[i], acc[i + 1]);
+            }
+            mn = fminf(mn, acc[E - 1]);
+            mx = fmaxf(mx, acc[E - 1]);
+            group_minmax_f32(mn, mx, L, red32);
+            const BlockQ b2 = block_q<B2>(mn, mx);
+            const bool clamp2 = __any_sync(0xffffffffu, top_code_overflows(mx, b2));
+            if (valid) {
+                const bool store2 = a.write_step2 != 0;
+                if (clamp2)
+                    sum_body<T, B2, NC, true>(acc, b2, y, store2, a.step2, e, leader, k);
+                else
+                    sum_body<T, B2, NC, false>(acc, b2, y, store2, a.step2, e, leader, k);
+            }
         }
     }
 }

@@ -193,7 +193,7 @@ __global__ void __launch_bounds__(FC_THREADS) k_ag(const AgArgs a)
 template <class T, int BITS> cudaError_t launch_quantize(const QuantArgs& a, cudaStream_t st);
 template <int BITS, int P> cudaError_t launch_rs(const RsArgs& a, cudaStream_t st);
 template <class T, int BITS> cudaError_t launch_ag(const AgArgs& a, cudaStream_t st);
-template <class T, int BITS, int P> cudaError_t launch_fused(const FusedArgs& a, cudaStream_t st);
+template <class T, int B1, int B2, int P> cudaError_t launch_fused(const FusedArgs& a, cudaStream_t st);
 
 // Persistent grid: enough CTAs of `threads` threads to fill every SM at the
 // kernel's occupancy, never more than there are tiles of `tile` elements.

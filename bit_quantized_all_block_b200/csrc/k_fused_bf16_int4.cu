@@ -1,13 +1,13 @@
-// Instantiations of the fused all-reduce kernel for __nv_bfloat16, INT4, P = 1..8.
+// Instantiations of the fused all-reduce kernel: __nv_bfloat16, INT4 in both steps, P = 1..8.
 #include "fc_launch_impl.cuh"
 
 namespace fc {
-template cudaError_t launch_fused<__nv_bfloat16, 4, 1>(const FusedArgs&, cudaStream_t);
-template cudaError_t launch_fused<__nv_bfloat16, 4, 2>(const FusedArgs&, cudaStream_t);
-template cudaError_t launch_fused<__nv_bfloat16, 4, 3>(const FusedArgs&, cudaStream_t);
-template cudaError_t launch_fused<__nv_bfloat16, 4, 4>(const FusedArgs&, cudaStream_t);
-template cudaError_t launch_fused<__nv_bfloat16, 4, 5>(const FusedArgs&, cudaStream_t);
-template cudaError_t launch_fused<__nv_bfloat16, 4, 6>(const FusedArgs&, cudaStream_t);
-template cudaError_t launch_fused<__nv_bfloat16, 4, 7>(const FusedArgs&, cudaStream_t);
-template cudaError_t launch_fused<__nv_bfloat16, 4, 8>(const FusedArgs&, cudaStream_t);
+template cudaError_t launch_fused<__nv_bfloat16, 4, 4, 1>(const FusedArgs&, cudaStream_t);
+template cudaError_t launch_fused<__nv_bfloat16, 4, 4, 2>(const FusedArgs&, cudaStream_t);
+template cudaError_t launch_fused<__nv_bfloat16, 4, 4, 3>(const FusedArgs&, cudaStream_t);
+template cudaError_t launch_fused<__nv_bfloat16, 4, 4, 4>(const FusedArgs&, cudaStream_t);
+template cudaError_t launch_fused<__nv_bfloat16, 4, 4, 5>(const FusedArgs&, cudaStream_t);
+template cudaError_t launch_fused<__nv_bfloat16, 4, 4, 6>(const FusedArgs&, cudaStream_t);
+template cudaError_t launch_fused<__nv_bfloat16, 4, 4, 7>(const FusedArgs&, cudaStream_t);
+template cudaError_t launch_fused<__nv_bfloat16, 4, 4, 8>(const FusedArgs&, cudaStream_t);
 }  // namespace fc

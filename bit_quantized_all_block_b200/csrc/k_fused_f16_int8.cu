@@ -1,13 +1,13 @@
-// Instantiations of the fused all-reduce kernel for __half, INT8, P = 1..8.
+// Instantiations of the fused all-reduce kernel: __half, INT8 in both steps, P = 1..8.
 #include "fc_launch_impl.cuh"
 
 namespace fc {
-template cudaError_t launch_fused<__half, 8, 1>(const FusedArgs&, cudaStream_t);
-template cudaError_t launch_fused<__half, 8, 2>(const FusedArgs&, cudaStream_t);
-template cudaError_t launch_fused<__half, 8, 3>(const FusedArgs&, cudaStream_t);
-template cudaError_t launch_fused<__half, 8, 4>(const FusedArgs&, cudaStream_t);
-template cudaError_t launch_fused<__half, 8, 5>(const FusedArgs&, cudaStream_t);
-template cudaError_t launch_fused<__half, 8, 6>(const FusedArgs&, cudaStream_t);
-template cudaError_t launch_fused<__half, 8, 7>(const FusedArgs&, cudaStream_t);
-template cudaError_t launch_fused<__half, 8, 8>(const FusedArgs&, cudaStream_t);
+template cudaError_t launch_fused<__half, 8, 8, 1>(const FusedArgs&, cudaStream_t);
+template cudaError_t launch_fused<__half, 8, 8, 2>(const FusedArgs&, cudaStream_t);
+template cudaError_t launch_fused<__half, 8, 8, 3>(const FusedArgs&, cudaStream_t);
+template cudaError_t launch_fused<__half, 8, 8, 4>(const FusedArgs&, cudaStream_t);
+template cudaError_t launch_fused<__half, 8, 8, 5>(const FusedArgs&, cudaStream_t);
+template cudaError_t launch_fused<__half, 8, 8, 6>(const FusedArgs&, cudaStream_t);
+template cudaError_t launch_fused<__half, 8, 8, 7>(const FusedArgs&, cudaStream_t);
+template cudaError_t launch_fused<__half, 8, 8, 8>(const FusedArgs&, cudaStream_t);
 }  // namespace fc

@@ -14,7 +14,8 @@
  * Arithmetic (the page gives no formulas; these are the plainest readings).
  * For a block of B values v_i (fp32; fp16/bf16 inputs are widened exactly),
  * at b bits with qmax = 2^b - 1, every operation binary32, round to nearest
- * even, no fused multiply-add:
+ * even; rne(a*b) rounds the exact product to the nearest integer (ties to
+ * even) in one step, and no other operation is fused:
  *   mn = min(0, v_i)   mx = max(0, v_i)
  *   s  = (mx == mn) ? 1 : (mx - mn) / qmax      inv = 1 / s
  *   z  = clamp(rne(-mn * inv), 0, qmax)          (uint8 zero-point)
@@ -87,14 +88,15 @@ typedef struct {
  * Errors: FC_ERR_INVALID_ARG for bad bits/block, n % block != 0, NULL outputs. */
 fc_status fc_payload_sizes(size_t n, int bits, int block, size_t* code_bytes, size_t* n_blocks);
 
-/* Step 1 on one rank (page: TL;DR, low-bit activation quantization; Fig. 4,
+/* Step 1 on one rank (page: TL;DR, activations quantized to low bit widths; Fig. 4,
  * per-block granularity): quantize the n fp16/bf16 values at x (device) into
  * the payload *out (device buffers).  Requires n % block == 0. */
 fc_status fc_quantize(const void* x, fc_dtype dtype, size_t n, int bits, int block,
                       const fc_qbuf* out, void* stream);
 
-/* Step 2, reduce-scatter (page: two-step All-Reduce; Fig. 5 right, "before
- * Reduce-Scatter"): in[0..P-1] are the P ranks' step-1 payloads of n elements
+/* Step 2, reduce-scatter (page: TL;DR, the first of the two all-reduce steps;
+ * Fig. 5 right, the quantization before the reduce-scatter): in[0..P-1] are
+ * the P ranks' step-1 payloads of n elements
  * each (host array of P structs of device pointers).  For every chunk c, the
  * owner's work is done: dequantize chunk c from all P payloads, sum in fp32 in
  * rank order 0..P-1, requantize.  *out receives the step-2 payload of all n
@@ -103,14 +105,15 @@ fc_status fc_quantize(const void* x, fc_dtype dtype, size_t n, int bits, int blo
 fc_status fc_rs_dequant_sum_requant(const fc_qbuf* in, int P, size_t n, int bits, int block,
                                     const fc_qbuf* out, void* stream);
 
-/* Step 3, all-gather (page: Fig. 5 right, "before All-Gather"): dequantize the
+/* Step 3, all-gather (page: Fig. 5 right, the quantization before the
+ * all-gather): dequantize the
  * gathered step-2 payload *in (n elements) and round each value to out_dtype
  * into y (device, n elements).  Requires n % block == 0. */
 fc_status fc_ag_dequant(const fc_qbuf* in, size_t n, int bits, int block, fc_dtype out_dtype,
                         void* y, void* stream);
 
-/* The fused all-reduce (page: TL;DR, "a fused CUDA kernel implements the
- * approach"): x is a host array of P device pointers, each to n fp16/bf16
+/* The fused all-reduce (page: TL;DR, the method runs as one fused CUDA
+ * kernel): x is a host array of P device pointers, each to n fp16/bf16
  * values (rank r's partial).  Writes the all-reduced result, rounded to dtype,
  * to y (device, n elements) in one kernel, without materialising the wire
  * payloads.  When step1 is non-NULL it is a host array of P payloads that
@@ -120,6 +123,24 @@ fc_status fc_ag_dequant(const fc_qbuf* in, size_t n, int bits, int block, fc_dty
 fc_status fc_quantized_allreduce(const void* const* x, int P, fc_dtype dtype, size_t n, int bits,
                                  int block, void* y, const fc_qbuf* step1, const fc_qbuf* step2,
                                  void* stream);
+
+/* The fused all-reduce with a width per step (page: Fig. 5 right compares the
+ * quantization error of the reduce-scatter step with that of the all-gather
+ * step).  bits_rs and bits_ag
+ * are each 4, 8 or 16; 16 means that step exchanges the fp16/bf16 values
+ * unquantized:
+ *   bits_rs == 16: the reduce-scatter sums the exactly widened inputs;
+ *   bits_ag == 16: the all-gather exchanges the fp32 sum rounded (nearest
+ *                  even) to dtype, which is then the output.
+ * step1 (P payloads of bits_rs) / step2 (one payload of bits_ag) are optional
+ * outputs as for fc_quantized_allreduce, and must be NULL for a step of width
+ * 16 (else FC_ERR_INVALID_ARG).  Equal quantized widths are provided for every
+ * P in [1, 8]; other combinations for P in {2, 4, 8} (FC_ERR_UNSUPPORTED for
+ * the rest).  fc_quantized_allreduce(.., bits, ..) is this call with
+ * bits_rs == bits_ag == bits.  Requires n % (P*block) == 0. */
+fc_status fc_quantized_allreduce_ex(const void* const* x, int P, fc_dtype dtype, size_t n, int bits_rs,
+                                    int bits_ag, int block, void* y, const fc_qbuf* step1,
+                                    const fc_qbuf* step2, void* stream);
 
 /* Static description of a status code. */
 const char* fc_status_string(fc_status status);

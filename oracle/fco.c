@@ -164,8 +164,8 @@ static uint16_t store_elem(float v, int dtype)
 }
 
 /* ------------------------------------------------------------------------ */
-/* Per-block asymmetric quantizer (page: TL;DR "low-bit activation           */
-/* quantization"; Fig. 4 block granularity along hidden).                    */
+/* Per-block asymmetric quantizer (page: TL;DR, activations are quantized   */
+/* to low bit widths; Fig. 4, block granularity along hidden).               */
 /* ------------------------------------------------------------------------ */
 
 /* Nearest integer, ties to even, of the exact product a*b of two fp32 values.
@@ -395,8 +395,9 @@ int fco_allreduce(const uint16_t* const* x, int P, int dtype, size_t n, int bits
 }
 
 /* ------------------------------------------------------------------------ */
-/* Per-step precision (page: Fig. 5 right, "MSE of quantization before       */
-/* Reduce-Scatter (RS) vs. All-Gather (AG)").  bits_rs and bits_ag are each  */
+/* Per-step precision (page: Fig. 5 right compares the quantization error   */
+/* of the reduce-scatter step with that of the all-gather step).  bits_rs    */
+/* and bits_ag are each                                                      */
 /* 4, 8 or 16; 16 means that step sends the 16-bit values unquantized:        */
 /*   bits_rs == 16: the RS sums the exactly widened inputs x_r;              */
 /*   bits_ag == 16: the AG sends the fp32 sum rounded to fp16/bf16, so the    */
