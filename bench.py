@@ -215,6 +215,56 @@ def run_reference(args, w):
     print(json.dumps(line), flush=True)
 
 
+def run_precision_sweep(args, w):
+    """Per-step precision (Fig. 5 right of the page): every width pair on one
+    GPU, timed like the main bench, with the MSE of each against the fp32 sum."""
+    import torch
+
+    import bit_quantized_all_block_b200 as fc
+
+    torch.cuda.set_device(0)
+    xs_host = synth.workload_partials(w)
+    tdt = torch.float16 if w.dtype == synth.FP16 else torch.bfloat16
+    xs = [torch.from_numpy(x.view(np.int16)).view(tdt).cuda() for x in xs_host]
+    S = xs[0].float()
+    for x in xs[1:]:
+        S = S + x.float()                        # fp32, rank order
+    S64 = S.double()
+    y = torch.empty(w.n, dtype=tdt, device="cuda")
+    for b1 in (16, 8, 4):
+        for b2 in (16, 8, 4):
+            s1 = [fc.QBuf.empty(w.n, b1, w.block) for _ in range(w.P)] if b1 != 16 else None
+            s2 = fc.QBuf.empty(w.n, b2, w.block) if b2 != 16 else None
+
+            def step():
+                fc.fc_quantized_allreduce_ex(xs, b1, b2, w.block, y=y, step1=s1, step2=s2)
+
+            for _ in range(args.warmup):
+                step()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(args.steps):
+                step()
+            e1.record()
+            torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1) / args.steps
+            err = y.double() - S64
+            mse = float((err * err).mean())
+            w1 = w.n * b1 // 8 + 5 * (w.n // w.block) if b1 != 16 else 0
+            w2 = w.n * b2 // 8 + 5 * (w.n // w.block) if b2 != 16 else 0
+            alg = w.P * w.n * 2 + w.n * 2 + w.P * w1 + w2
+            print(json.dumps({
+                "metric": METRIC, "mode": "precision_sweep", "workload": w.name,
+                "bits_rs": b1, "bits_ag": b2, "us": round(ms * 1e3, 2),
+                "input_gbs": round(w.P * w.n * 2 / (ms * 1e-3) / 1e9, 1),
+                "achieved_gbs": round(alg / (ms * 1e-3) / 1e9, 1),
+                "mse_vs_fp32_sum": mse, "rel_mse": mse / float((S64 * S64).mean()),
+                "wire_bytes_per_rank": (w1 if b1 != 16 else w.n * 2) + (w2 if b2 != 16 else w.n * 2)}),
+                flush=True)
+            del s1, s2
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -229,11 +279,16 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=0,
                     help="token rows per rank for the cpu_baseline sample (0 = the whole workload)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--precision-sweep", action="store_true",
+                    help="time the fused kernel for every (RS bits, AG bits) in {4,8,16}^2 on the "
+                         "workload and report each variant's MSE (one JSON line per variant)")
     args = ap.parse_args()
     assert args.warmup >= 3 or args.impl == "reference", "at least 3 warm-up steps"
     w = WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, w)
+    if args.precision_sweep:
+        return run_precision_sweep(args, w)
 
     import torch
     import torch.distributed as dist
