@@ -344,7 +344,26 @@ def main():
     with ClockSampler(local) as clocks:
         barrier()
         torch.cuda.synchronize()
-        if not small:
+        if args.variant == "staged":
+            # events between the stages give each staged kernel its own time
+            marks = []
+            for _ in range(args.steps):
+                if small:
+                    flush.zero_()
+                ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+                ev[0].record(stream)
+                for r in range(w.P):
+                    fc.fc_quantize(xs[r], w.bits, w.block, out=s1[r])
+                ev[1].record(stream)
+                fc.fc_rs_dequant_sum_requant(s1, w.bits, w.block, out=s2)
+                ev[2].record(stream)
+                fc.fc_ag_dequant(s2, tdt, y=y)
+                ev[3].record(stream)
+                marks.append(ev)
+            torch.cuda.synchronize()
+            stage_ms = [sum(m[i].elapsed_time(m[i + 1]) for m in marks) / args.steps for i in range(3)]
+            ms = sum(stage_ms)
+        elif not small:
             ev0.record(stream)
             for _ in range(args.steps):
                 step()
@@ -414,6 +433,16 @@ def main():
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks.summary(),
     }
+
+    if args.variant == "staged":
+        w2b = payload_bytes(w)
+        per = {"k_quantize (x P)": (stage_ms[0], w.P * (w.n * 2 + w2b)),
+               "k_rs": (stage_ms[1], w.P * w2b + w2b),
+               "k_ag": (stage_ms[2], w2b + w.n * 2)}
+        line["kernels"] = {k: {"us": round(t * 1e3, 2), "algorithmic_bytes": b,
+                               "achieved_gbs": round(b / (t * 1e-3) / 1e9, 1),
+                               "frac": round(b / (t * 1e-3) / 1e9 / peak, 4)}
+                           for k, (t, b) in per.items()}
 
     # ---- result quality and the CPU baseline (rank 0, N = 1 only) -----------
     if rank == 0:

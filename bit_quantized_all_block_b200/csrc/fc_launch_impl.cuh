@@ -1,7 +1,7 @@
 // fc_launch_impl.cuh -- launcher bodies, included by the instantiation units.
 #pragma once
 
-#include "fc_fused.cuh"
+#include "fc_staged.cuh"
 
 namespace fc {
 
@@ -9,10 +9,10 @@ template <class T, int BITS>
 cudaError_t launch_quantize(const QuantArgs& a, cudaStream_t st)
 {
     int grid = 0;
-    cudaError_t e = persistent_grid((const void*)k_quantize<T, BITS>, FC_THREADS, a.n, FC_TILE, &grid);
+    cudaError_t e = persistent_grid((const void*)k_quantize<T, BITS>, ST_THREADS, a.n, QuantShape::TILE, &grid);
     if (e != cudaSuccess)
         return e;
-    k_quantize<T, BITS><<<grid, FC_THREADS, 0, st>>>(a);
+    k_quantize<T, BITS><<<grid, ST_THREADS, 0, st>>>(a);
     return cudaGetLastError();
 }
 
@@ -20,10 +20,10 @@ template <int BITS, int P>
 cudaError_t launch_rs(const RsArgs& a, cudaStream_t st)
 {
     int grid = 0;
-    cudaError_t e = persistent_grid((const void*)k_rs<BITS, P>, FC_THREADS, a.n, FC_TILE, &grid);
+    cudaError_t e = persistent_grid((const void*)k_rs<BITS, P>, ST_THREADS, a.n, RsShape<P>::TILE, &grid);
     if (e != cudaSuccess)
         return e;
-    k_rs<BITS, P><<<grid, FC_THREADS, 0, st>>>(a);
+    k_rs<BITS, P><<<grid, ST_THREADS, 0, st>>>(a);
     return cudaGetLastError();
 }
 
@@ -31,10 +31,10 @@ template <class T, int BITS>
 cudaError_t launch_ag(const AgArgs& a, cudaStream_t st)
 {
     int grid = 0;
-    cudaError_t e = persistent_grid((const void*)k_ag<T, BITS>, FC_THREADS, a.n, FC_TILE, &grid);
+    cudaError_t e = persistent_grid((const void*)k_ag<T, BITS>, ST_THREADS, a.n, AgShape::TILE, &grid);
     if (e != cudaSuccess)
         return e;
-    k_ag<T, BITS><<<grid, FC_THREADS, 0, st>>>(a);
+    k_ag<T, BITS><<<grid, ST_THREADS, 0, st>>>(a);
     return cudaGetLastError();
 }
 

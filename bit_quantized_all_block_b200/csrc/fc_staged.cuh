@@ -1,0 +1,273 @@
+// fc_staged.cuh -- the staged kernels: the three steps of the two-step
+// quantized all-reduce as separate launches with the payloads in HBM between
+// them (Flash Communication, sciencestack.ai/paper/2412.04964: TL;DR, the
+// quantize -> reduce-scatter -> all-gather structure; Fig. 5 right).
+//
+//   k_quantize<T, BITS>   x_r -> step-1 payload (one rank)
+//   k_rs<BITS, P>         P step-1 payloads -> step-2 payload (all chunks)
+//   k_ag<T, BITS>         step-2 payload -> y
+//
+// Same layout as the fused kernel (fc_fused.cuh): 256-thread persistent CTAs,
+// each thread owns E contiguous elements (one base pointer, immediate
+// offsets, 128-bit accesses), a block is L = B/E consecutive threads that
+// reduce min/max by xor-shuffles (and shared memory beyond a warp), the next
+// tile's inputs are loaded as soon as the current ones are consumed, codes
+// are rounded by one FMA, and the rarely binding upper clamp runs behind a
+// warp-uniform branch.
+#pragma once
+
+#include "fc_fused.cuh"
+
+namespace fc {
+
+constexpr int ST_THREADS = 256;
+
+template <int NC_>
+struct StShape {
+    static constexpr int NC = NC_;
+    static constexpr int E = NC * FC_CHUNK;
+    static constexpr int TILE = ST_THREADS * E;
+};
+using QuantShape = StShape<4>;                          // 32 elements per thread
+using AgShape = StShape<4>;
+template <int P> using RsShape = StShape<(P <= 4 ? 4 : 2)>;
+
+// Load a thread's E codes (E*BITS/8 contiguous bytes) at element offset e.
+template <int BITS, int NC>
+__device__ __forceinline__ void load_thread_codes(const uint8_t* codes, size_t e, uint32_t* w)
+{
+    constexpr int NW = NC * BITS / 4;
+    const uint8_t* p = codes + e * BITS / 8;
+    if constexpr (NW % 4 == 0) {
+#pragma unroll
+        for (int i = 0; i < NW; i += 4) {
+            const uint4 v = ld_nc(p + 4 * i);
+            w[i] = v.x;
+            w[i + 1] = v.y;
+            w[i + 2] = v.z;
+            w[i + 3] = v.w;
+        }
+    } else {
+        const uint2 v = ld_stream_u2(p);
+        w[0] = v.x;
+        w[1] = v.y;
+    }
+}
+
+// Shifted codes of chunk c of a thread's code words.
+template <int BITS>
+__device__ __forceinline__ void chunk_shifted(const uint32_t* w, int c, float* sh)
+{
+    if constexpr (BITS == 8)
+        unpack_chunk<8>(w + 2 * c, sh);
+    else
+        unpack_chunk<4>(w + c, sh);
+}
+
+// Block extremes (0 folded in) of E fp32 values held by each of L threads.
+template <int E>
+__device__ __forceinline__ void block_minmax_f32(const float* v, int L, float2* red, float& mn, float& mx)
+{
+    mn = fminf(v[0], 0.0f);
+    mx = fmaxf(v[0], 0.0f);
+#pragma unroll
+    for (int i = 1; i + 1 < E; i += 2) {
+        mn = min3(mn, v[i], v[i + 1]);
+        mx = max3(mx, v[i], v[i + 1]);
+    }
+    mn = fminf(mn, v[E - 1]);
+    mx = fmaxf(mx, v[E - 1]);
+    group_minmax_f32(mn, mx, L, red);
+}
+
+// Quantize E fp32 values (one thread's share of a block) and store codes,
+// scale and zero-point.
+template <int BITS, int NC, bool CLAMP>
+__device__ __forceinline__ void quant_store(const float* v, const BlockQ& b, const QPtr& out, size_t e,
+                                            bool leader, size_t k)
+{
+    const float cqz = __fsub_rn(b.cq, b.zf);
+    uint32_t words[NC * BITS / 4];
+#pragma unroll
+    for (int c = 0; c < NC; c++) {
+        float sh[8];
+#pragma unroll
+        for (int i = 0; i < 8; i++) {
+            float r = round_product_shifted(v[c * 8 + i], b.inv);
+            if (CLAMP)
+                r = fminf(r, cqz);
+            sh[i] = __fadd_rn(r, b.zf);
+        }
+        pack_chunk<BITS>(sh, words, c);
+    }
+    store_thread_codes<BITS, NC>(out.codes, e, words);
+    if (leader) {
+        out.scales[k] = b.s;
+        out.zps[k] = zp_byte(b);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Step 1 on one rank.
+template <class T, int BITS>
+__global__ void __launch_bounds__(ST_THREADS) k_quantize(const QuantArgs a)
+{
+    using P2 = Pair<T>;
+    using T2 = typename P2::T2;
+    constexpr int NC = QuantShape::NC, E = QuantShape::E, TILE = QuantShape::TILE;
+    __shared__ uint32_t red[ST_THREADS / 32];
+    const int L = a.block / E;
+    const int j = threadIdx.x % L;
+    const int lg_block = __ffs(a.block) - 1;
+    const size_t toff = (size_t)threadIdx.x * E;
+    const size_t stride = (size_t)gridDim.x * TILE;
+    const T* x = static_cast<const T*>(a.x);
+
+    uint4 raw[NC];
+    {
+        const size_t e0 = (size_t)blockIdx.x * TILE + toff;
+        if (e0 < a.n) {
+            load_chunks<T, NC>(raw, x + e0);
+        } else {
+#pragma unroll
+            for (int c = 0; c < NC; c++)
+                raw[c] = make_uint4(0, 0, 0, 0);
+        }
+    }
+    for (size_t base = (size_t)blockIdx.x * TILE; base < a.n; base += stride) {
+        const size_t e = base + toff;
+        const bool valid = e < a.n;
+        const size_t k = e >> lg_block;
+        const T2 t = as_t2<T2>(group_min_negmax<T>(local_min_negmax<T, NC>(raw), L, red));
+        const float mx = fmaxf(-P2::hi(t), 0.0f);
+        const BlockQ b = block_q<BITS>(fminf(P2::lo(t), 0.0f), mx);
+        const bool clamp = __any_sync(0xffffffffu, top_code_overflows(mx, b));
+        float v[E];
+#pragma unroll
+        for (int c = 0; c < NC; c++) {
+            const uint32_t w[4] = {raw[c].x, raw[c].y, raw[c].z, raw[c].w};
+#pragma unroll
+            for (int h = 0; h < 4; h++) {
+                const float2 f = P2::to_f2(as_t2<T2>(w[h]));
+                v[c * 8 + 2 * h] = f.x;
+                v[c * 8 + 2 * h + 1] = f.y;
+            }
+        }
+        if (e + stride < a.n)
+            load_chunks<T, NC>(raw, x + e + stride);
+        if (valid) {
+            if (clamp)
+                quant_store<BITS, NC, true>(v, b, a.out, e, j == 0, k);
+            else
+                quant_store<BITS, NC, false>(v, b, a.out, e, j == 0, k);
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Step 2 (reduce-scatter) for every chunk at once: chunk ownership does not
+// change the arithmetic, since chunks are block-aligned and each block of the
+// sum depends only on the same block of every rank.
+template <int BITS, int P>
+__global__ void __launch_bounds__(ST_THREADS) k_rs(const RsArgs a)
+{
+    constexpr int NC = RsShape<P>::NC, E = RsShape<P>::E, TILE = RsShape<P>::TILE;
+    constexpr int NW = NC * BITS / 4;
+    __shared__ float2 red[ST_THREADS / 32];
+    const int L = a.block / E;
+    const int j = threadIdx.x % L;
+    const int lg_block = __ffs(a.block) - 1;
+    const size_t toff = (size_t)threadIdx.x * E;
+    const size_t stride = (size_t)gridDim.x * TILE;
+
+    uint32_t w[P][NW];
+    float s[P], mz[P];
+    {
+        const size_t e0 = (size_t)blockIdx.x * TILE + toff;
+        const size_t k0 = e0 >> lg_block;
+#pragma unroll
+        for (int r = 0; r < P; r++) {
+            if (e0 < a.n) {
+                load_thread_codes<BITS, NC>(a.in[r].codes, e0, w[r]);
+                s[r] = a.in[r].scales[k0];
+                mz[r] = __uint_as_float(FC_MAGIC_BITS + a.in[r].zps[k0]);
+            } else {
+#pragma unroll
+                for (int i = 0; i < NW; i++)
+                    w[r][i] = 0;
+                s[r] = 1.0f;
+                mz[r] = FC_MAGIC;
+            }
+        }
+    }
+    for (size_t base = (size_t)blockIdx.x * TILE; base < a.n; base += stride) {
+        const size_t e = base + toff;
+        const bool valid = e < a.n;
+        const bool valid_next = e + stride < a.n;
+        const size_t k = e >> lg_block;
+        const size_t kn = (e + stride) >> lg_block;
+        float acc[E];
+#pragma unroll
+        for (int r = 0; r < P; r++) {
+#pragma unroll
+            for (int c = 0; c < NC; c++) {
+                float sh[8];
+                chunk_shifted<BITS>(w[r], c, sh);
+#pragma unroll
+                for (int i = 0; i < 8; i++) {
+                    const float xh = __fmul_rn(__fsub_rn(sh[i], mz[r]), s[r]);
+                    acc[c * 8 + i] = (r == 0) ? xh : __fadd_rn(acc[c * 8 + i], xh);
+                }
+            }
+            if (valid_next) {   // refill rank r with the next tile
+                load_thread_codes<BITS, NC>(a.in[r].codes, e + stride, w[r]);
+                s[r] = a.in[r].scales[kn];
+                mz[r] = __uint_as_float(FC_MAGIC_BITS + a.in[r].zps[kn]);
+            }
+        }
+        float mn, mx;
+        block_minmax_f32<E>(acc, L, red, mn, mx);
+        const BlockQ b = block_q<BITS>(mn, mx);
+        const bool clamp = __any_sync(0xffffffffu, top_code_overflows(mx, b));
+        if (valid) {
+            if (clamp)
+                quant_store<BITS, NC, true>(acc, b, a.out, e, j == 0, k);
+            else
+                quant_store<BITS, NC, false>(acc, b, a.out, e, j == 0, k);
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Step 3 (all-gather): dequantize to fp16/bf16.
+template <class T, int BITS>
+__global__ void __launch_bounds__(ST_THREADS) k_ag(const AgArgs a)
+{
+    constexpr int NC = AgShape::NC, E = AgShape::E, TILE = AgShape::TILE;
+    constexpr int NW = NC * BITS / 4;
+    const int lg_block = __ffs(a.block) - 1;
+    const size_t toff = (size_t)threadIdx.x * E;
+    const size_t stride = (size_t)gridDim.x * TILE;
+    T* y = static_cast<T*>(a.y);
+    for (size_t base = (size_t)blockIdx.x * TILE; base < a.n; base += stride) {
+        const size_t e = base + toff;
+        if (e >= a.n)
+            continue;
+        const size_t k = e >> lg_block;
+        uint32_t w[NW];
+        load_thread_codes<BITS, NC>(a.in.codes, e, w);
+        const float s = a.in.scales[k];
+        const float mz = __uint_as_float(FC_MAGIC_BITS + a.in.zps[k]);
+#pragma unroll
+        for (int c = 0; c < NC; c++) {
+            float sh[8], v[8];
+            chunk_shifted<BITS>(w, c, sh);
+#pragma unroll
+            for (int i = 0; i < 8; i++)
+                v[i] = __fmul_rn(__fsub_rn(sh[i], mz), s);
+            st_stream(y + e + c * FC_CHUNK, narrow8<T>(v));
+        }
+    }
+}
+
+}  // namespace fc
