@@ -272,7 +272,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
-    ap.add_argument("--variant", default="fused", choices=["fused", "fused_nopayload", "staged"])
+    ap.add_argument("--variant", default="fused",
+                    help="fused | fused_nopayload | staged, or a comma-separated list (one JSON line each)")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--ref-rows", type=int, default=256,
                     help="token rows per rank in one reference (oracle) step")
@@ -284,6 +285,8 @@ def main():
                          "workload and report each variant's MSE (one JSON line per variant)")
     args = ap.parse_args()
     assert args.warmup >= 3 or args.impl == "reference", "at least 3 warm-up steps"
+    for v in args.variant.split(","):
+        assert v in ("fused", "fused_nopayload", "staged"), f"unknown variant {v}"
     w = WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, w)
@@ -315,162 +318,164 @@ def main():
     s2 = fc.QBuf.empty(w.n, w.bits, w.block)
     stream = torch.cuda.current_stream()
 
-    def step():
-        if args.variant == "fused":
-            fc.fc_quantized_allreduce(xs, w.bits, w.block, y=y, step1=s1, step2=s2)
-        elif args.variant == "fused_nopayload":
-            fc.fc_quantized_allreduce(xs, w.bits, w.block, y=y)
-        else:
-            for r in range(w.P):
-                fc.fc_quantize(xs[r], w.bits, w.block, out=s1[r])
-            fc.fc_rs_dequant_sum_requant(s1, w.bits, w.block, out=s2)
-            fc.fc_ag_dequant(s2, tdt, y=y)
-
-    launches_per_step = 1 if args.variant.startswith("fused") else w.P + 2
-
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-
-    # ---- timed region: K steps, events on the launching stream ---------------
-    # Workloads larger than L2 run back to back (every step streams from HBM).
-    # Smaller ones flush L2 with a 512 MB write before every step and time each
-    # step with its own pair of events (the flush keeps the GPU busy while the
-    # host enqueues the step, so no host gap falls inside the pair).
-    step_bytes = algorithmic_bytes(w, args.variant)
-    small = step_bytes < L2_FLUSH_THRESHOLD
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda") if small else None
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local) as clocks:
-        barrier()
-        torch.cuda.synchronize()
-        if args.variant == "staged":
-            # events between the stages give each staged kernel its own time
-            marks = []
-            for _ in range(args.steps):
-                if small:
-                    flush.zero_()
-                ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
-                ev[0].record(stream)
+    variants = args.variant.split(",")
+    for vi, variant in enumerate(variants):
+        def step():
+            if variant == "fused":
+                fc.fc_quantized_allreduce(xs, w.bits, w.block, y=y, step1=s1, step2=s2)
+            elif variant == "fused_nopayload":
+                fc.fc_quantized_allreduce(xs, w.bits, w.block, y=y)
+            else:
                 for r in range(w.P):
                     fc.fc_quantize(xs[r], w.bits, w.block, out=s1[r])
-                ev[1].record(stream)
                 fc.fc_rs_dequant_sum_requant(s1, w.bits, w.block, out=s2)
-                ev[2].record(stream)
                 fc.fc_ag_dequant(s2, tdt, y=y)
-                ev[3].record(stream)
-                marks.append(ev)
-            torch.cuda.synchronize()
-            stage_ms = [sum(m[i].elapsed_time(m[i + 1]) for m in marks) / args.steps for i in range(3)]
-            ms = sum(stage_ms)
-        elif not small:
-            ev0.record(stream)
-            for _ in range(args.steps):
-                step()
-            ev1.record(stream)
-            torch.cuda.synchronize()
-            ms = ev0.elapsed_time(ev1) / args.steps
-        else:
-            pairs = []
-            for _ in range(args.steps):
-                flush.zero_()
-                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                a.record(stream)
-                step()
-                b.record(stream)
-                pairs.append((a, b))
-            torch.cuda.synchronize()
-            ms = sum(a.elapsed_time(b) for a, b in pairs) / args.steps
-        barrier()
-    ms = max_over_ranks(ms, world)
 
-    # ---- end to end through the public API with host buffers -----------------
-    y_host = torch.empty(w.n, dtype=tdt).pin_memory()
-    for _ in range(2):
-        for r in range(w.P):
-            xs[r].copy_(xs_pinned[r], non_blocking=True)
-        step()
-        y_host.copy_(y, non_blocking=True)
-    torch.cuda.synchronize()
-    barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.e2e_steps):
-        for r in range(w.P):
-            xs[r].copy_(xs_pinned[r], non_blocking=True)
-        step()
-        y_host.copy_(y, non_blocking=True)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    ms_e2e = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, world)
+        launches_per_step = 1 if variant.startswith("fused") else w.P + 2
 
-    in_bytes = w.P * w.n * 2
-    value = job_throughput(in_bytes, world, ms)
-    value_e2e = job_throughput(in_bytes, world, ms_e2e)
-    alg = algorithmic_bytes(w, args.variant)
-    peak, peak_kind = read_peak()
-    achieved = alg / (ms * 1e-3) / 1e9
-    traffic = read_traffic(w.name, args.variant)
-
-    line = {
-        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
-        "us_per_allreduce": round(ms * 1e3, 2),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "f32", "data": "synthetic",
-        "config": {"workload": w.name, "description": w.describe(), "variant": args.variant,
-                   "parallelism": f"replicas x{world} (P={w.P} ranks emulated per GPU)",
-                   "l2": (f"L2 flushed (512 MB write) before each step, each step timed alone"
-                          if small else
-                          f"inputs larger than L2 ({in_bytes / 1e6:.0f} MB read per step), no flush")},
-        "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
-                     "frac": round(achieved / peak, 4), "traffic": traffic,
-                     "peak_kind": f"{peak_kind} copy bandwidth",
-                     "algorithmic_bytes_per_launch": alg if args.variant.startswith("fused") else None,
-                     "algorithmic_bytes_per_step": alg},
-        "e2e": {"value": round(value_e2e, 3), "unit": "GB/s", "h2d_bytes_per_step": in_bytes,
-                "d2h_bytes_per_step": w.n * 2},
-        "gpu_launches": launches_per_step * args.steps,
-        "clocks": clocks.summary(),
-    }
-
-    if args.variant == "staged":
-        w2b = payload_bytes(w)
-        per = {"k_quantize (x P)": (stage_ms[0], w.P * (w.n * 2 + w2b)),
-               "k_rs": (stage_ms[1], w.P * w2b + w2b),
-               "k_ag": (stage_ms[2], w2b + w.n * 2)}
-        line["kernels"] = {k: {"us": round(t * 1e3, 2), "algorithmic_bytes": b,
-                               "achieved_gbs": round(b / (t * 1e-3) / 1e9, 1),
-                               "frac": round(b / (t * 1e-3) / 1e9 / peak, 4)}
-                           for k, (t, b) in per.items()}
-
-    # ---- result quality and the CPU baseline (rank 0, N = 1 only) -----------
-    if rank == 0:
+        for _ in range(args.warmup):
+            step()
         torch.cuda.synchronize()
-        y_np = y.view(torch.int16).cpu().numpy().view(np.uint16)
-        import torch as _t
-        wide = [_t.from_numpy(x.view(np.int16)).view(tdt).to(_t.float32).numpy() for x in xs_host]
-        S = wide[0].copy()
-        for v in wide[1:]:
-            S += v                                      # fp32, rank order 0..P-1
-        yf = _t.from_numpy(y_np.view(np.int16)).view(tdt).to(_t.float32).numpy().astype(np.float64)
-        err = yf - S.astype(np.float64)
-        mse = float(np.mean(err * err))
-        line["quality"] = {"mse_vs_fp32_sum": mse,
-                           "rel_mse": mse / float(np.mean(S.astype(np.float64) ** 2))}
-        if world == 1 and not args.no_cpu_baseline:
-            import oracle
-            rows = args.cpu_rows or w.T
-            sub = [x[: rows * w.H] for x in xs_host]
-            t0 = time.perf_counter()
-            y_ref, _, _ = oracle.allreduce(sub, w.dtype, w.bits, w.block)
-            dt = time.perf_counter() - t0
-            line["cpu_baseline"] = {
-                "value": round(sum(x.size for x in sub) * 2 / dt / 1e9, 5), "unit": "GB/s", "cores": 1,
-                "kind": "oracle",
-                "sample": f"{rows} of {w.T} token rows per rank, {dt:.1f} s, single thread"}
-            line["quality"]["bit_exact_vs_oracle"] = bool(np.array_equal(y_np[: rows * w.H], y_ref))
-        print(json.dumps(line), flush=True)
+
+        # ---- timed region: K steps, events on the launching stream ---------------
+        # Workloads larger than L2 run back to back (every step streams from HBM).
+        # Smaller ones flush L2 with a 512 MB write before every step and time each
+        # step with its own pair of events (the flush keeps the GPU busy while the
+        # host enqueues the step, so no host gap falls inside the pair).
+        step_bytes = algorithmic_bytes(w, variant)
+        small = step_bytes < L2_FLUSH_THRESHOLD
+        flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda") if small else None
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with ClockSampler(local) as clocks:
+            barrier()
+            torch.cuda.synchronize()
+            if variant == "staged":
+                # events between the stages give each staged kernel its own time
+                marks = []
+                for _ in range(args.steps):
+                    if small:
+                        flush.zero_()
+                    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+                    ev[0].record(stream)
+                    for r in range(w.P):
+                        fc.fc_quantize(xs[r], w.bits, w.block, out=s1[r])
+                    ev[1].record(stream)
+                    fc.fc_rs_dequant_sum_requant(s1, w.bits, w.block, out=s2)
+                    ev[2].record(stream)
+                    fc.fc_ag_dequant(s2, tdt, y=y)
+                    ev[3].record(stream)
+                    marks.append(ev)
+                torch.cuda.synchronize()
+                stage_ms = [sum(m[i].elapsed_time(m[i + 1]) for m in marks) / args.steps for i in range(3)]
+                ms = sum(stage_ms)
+            elif not small:
+                ev0.record(stream)
+                for _ in range(args.steps):
+                    step()
+                ev1.record(stream)
+                torch.cuda.synchronize()
+                ms = ev0.elapsed_time(ev1) / args.steps
+            else:
+                pairs = []
+                for _ in range(args.steps):
+                    flush.zero_()
+                    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    a.record(stream)
+                    step()
+                    b.record(stream)
+                    pairs.append((a, b))
+                torch.cuda.synchronize()
+                ms = sum(a.elapsed_time(b) for a, b in pairs) / args.steps
+            barrier()
+        ms = max_over_ranks(ms, world)
+
+        # ---- end to end through the public API with host buffers -----------------
+        y_host = torch.empty(w.n, dtype=tdt).pin_memory()
+        for _ in range(2):
+            for r in range(w.P):
+                xs[r].copy_(xs_pinned[r], non_blocking=True)
+            step()
+            y_host.copy_(y, non_blocking=True)
+        torch.cuda.synchronize()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            for r in range(w.P):
+                xs[r].copy_(xs_pinned[r], non_blocking=True)
+            step()
+            y_host.copy_(y, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms_e2e = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, world)
+
+        in_bytes = w.P * w.n * 2
+        value = job_throughput(in_bytes, world, ms)
+        value_e2e = job_throughput(in_bytes, world, ms_e2e)
+        alg = algorithmic_bytes(w, variant)
+        peak, peak_kind = read_peak()
+        achieved = alg / (ms * 1e-3) / 1e9
+        traffic = read_traffic(w.name, variant)
+
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
+            "us_per_allreduce": round(ms * 1e3, 2),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32", "data": "synthetic",
+            "config": {"workload": w.name, "description": w.describe(), "variant": variant,
+                       "parallelism": f"replicas x{world} (P={w.P} ranks emulated per GPU)",
+                       "l2": (f"L2 flushed (512 MB write) before each step, each step timed alone"
+                              if small else
+                              f"inputs larger than L2 ({in_bytes / 1e6:.0f} MB read per step), no flush")},
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
+                         "frac": round(achieved / peak, 4), "traffic": traffic,
+                         "peak_kind": f"{peak_kind} copy bandwidth",
+                         "algorithmic_bytes_per_launch": alg if variant.startswith("fused") else None,
+                         "algorithmic_bytes_per_step": alg},
+            "e2e": {"value": round(value_e2e, 3), "unit": "GB/s", "h2d_bytes_per_step": in_bytes,
+                    "d2h_bytes_per_step": w.n * 2},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clocks.summary(),
+        }
+
+        if variant == "staged":
+            w2b = payload_bytes(w)
+            per = {"k_quantize (x P)": (stage_ms[0], w.P * (w.n * 2 + w2b)),
+                   "k_rs": (stage_ms[1], w.P * w2b + w2b),
+                   "k_ag": (stage_ms[2], w2b + w.n * 2)}
+            line["kernels"] = {k: {"us": round(t * 1e3, 2), "algorithmic_bytes": b,
+                                   "achieved_gbs": round(b / (t * 1e-3) / 1e9, 1),
+                                   "frac": round(b / (t * 1e-3) / 1e9 / peak, 4)}
+                               for k, (t, b) in per.items()}
+
+        # ---- result quality and the CPU baseline (rank 0, N = 1 only) -----------
+        if rank == 0:
+            torch.cuda.synchronize()
+            y_np = y.view(torch.int16).cpu().numpy().view(np.uint16)
+            import torch as _t
+            wide = [_t.from_numpy(x.view(np.int16)).view(tdt).to(_t.float32).numpy() for x in xs_host]
+            S = wide[0].copy()
+            for v in wide[1:]:
+                S += v                                      # fp32, rank order 0..P-1
+            yf = _t.from_numpy(y_np.view(np.int16)).view(tdt).to(_t.float32).numpy().astype(np.float64)
+            err = yf - S.astype(np.float64)
+            mse = float(np.mean(err * err))
+            line["quality"] = {"mse_vs_fp32_sum": mse,
+                               "rel_mse": mse / float(np.mean(S.astype(np.float64) ** 2))}
+            if world == 1 and not args.no_cpu_baseline and vi == 0:
+                import oracle
+                rows = args.cpu_rows or w.T
+                sub = [x[: rows * w.H] for x in xs_host]
+                t0 = time.perf_counter()
+                y_ref, _, _ = oracle.allreduce(sub, w.dtype, w.bits, w.block)
+                dt = time.perf_counter() - t0
+                line["cpu_baseline"] = {
+                    "value": round(sum(x.size for x in sub) * 2 / dt / 1e9, 5), "unit": "GB/s", "cores": 1,
+                    "kind": "oracle",
+                    "sample": f"{rows} of {w.T} token rows per rank, {dt:.1f} s, single thread"}
+                line["quality"]["bit_exact_vs_oracle"] = bool(np.array_equal(y_np[: rows * w.H], y_ref))
+            print(json.dumps(line), flush=True)
 
     if world > 1:
         dist.destroy_process_group()
