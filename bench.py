@@ -280,6 +280,8 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=0,
                     help="token rows per rank for the cpu_baseline sample (0 = the whole workload)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="launch the timed steps one by one instead of replaying a CUDA graph of them")
     ap.add_argument("--precision-sweep", action="store_true",
                     help="time the fused kernel for every (RS bits, AG bits) in {4,8,16}^2 on the "
                          "workload and report each variant's MSE (one JSON line per variant)")
@@ -344,6 +346,15 @@ def main():
         # host enqueues the step, so no host gap falls inside the pair).
         step_bytes = algorithmic_bytes(w, variant)
         small = step_bytes < L2_FLUSH_THRESHOLD
+        graph = None
+        if not small and variant != "staged" and not args.no_graph:
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                for _ in range(args.steps):
+                    step()
+            torch.cuda.synchronize()
+            graph.replay()                      # one untimed replay
+            torch.cuda.synchronize()
         flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda") if small else None
         ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         with ClockSampler(local) as clocks:
@@ -369,9 +380,14 @@ def main():
                 stage_ms = [sum(m[i].elapsed_time(m[i + 1]) for m in marks) / args.steps for i in range(3)]
                 ms = sum(stage_ms)
             elif not small:
+                # the K steps are captured once in a CUDA graph and replayed, so
+                # host launch gaps do not enter the device time
                 ev0.record(stream)
-                for _ in range(args.steps):
-                    step()
+                if graph is not None:
+                    graph.replay()
+                else:
+                    for _ in range(args.steps):
+                        step()
                 ev1.record(stream)
                 torch.cuda.synchronize()
                 ms = ev0.elapsed_time(ev1) / args.steps
@@ -425,6 +441,7 @@ def main():
             "dtype": "f32", "data": "synthetic",
             "config": {"workload": w.name, "description": w.describe(), "variant": variant,
                        "parallelism": f"replicas x{world} (P={w.P} ranks emulated per GPU)",
+                       "launch": "CUDA graph of the timed steps" if graph is not None else "stream launches",
                        "l2": (f"L2 flushed (512 MB write) before each step, each step timed alone"
                               if small else
                               f"inputs larger than L2 ({in_bytes / 1e6:.0f} MB read per step), no flush")},

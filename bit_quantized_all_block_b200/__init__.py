@@ -67,8 +67,9 @@ def _lib():
         L.fc_ag_dequant.argtypes = [QP, S, I, I, I, P, P]
         L.fc_quantized_allreduce.argtypes = [ctypes.POINTER(P), I, I, S, I, I, P, QP, QP, P]
         L.fc_quantized_allreduce_ex.argtypes = [ctypes.POINTER(P), I, I, S, I, I, I, P, QP, QP, P]
+        L.fc_gemm_quantize.argtypes = [P, P, I, I, I, I, I, I, QP, P, P, P]
         for f in ("fc_payload_sizes", "fc_quantize", "fc_rs_dequant_sum_requant", "fc_ag_dequant",
-                  "fc_quantized_allreduce", "fc_quantized_allreduce_ex"):
+                  "fc_quantized_allreduce", "fc_quantized_allreduce_ex", "fc_gemm_quantize"):
             getattr(L, f).restype = I
         L.fc_status_string.argtypes = [I]
         L.fc_status_string.restype = ctypes.c_char_p
@@ -229,4 +230,33 @@ def fc_quantized_allreduce_ex(xs, bits_rs: int, bits_ag: int, block: int, y=None
                                             ctypes.byref(s2) if s2 is not None else None,
                                             _stream(stream)), "fc_quantized_allreduce_ex")
     return y
+
+
+def fc_gemm_quantize(a, w, bits: int, block: int, out: QBuf | None = None, partial=None, status=None,
+                     quantize: bool = True, stream=None):
+    """One rank's partial a @ w.T (tensor cores, fp32 accumulate, rounded to a.dtype) with the
+    step-1 quantizer fused into the epilogue.
+
+    Returns (payload or None, partial or None, status tensor).  ``quantize=False`` skips the
+    payload (plain GEMM writing the partial); pass ``partial`` to also receive the partial."""
+    import torch
+    M, K = a.shape
+    N, K2 = w.shape
+    if K != K2 or a.dtype != w.dtype:
+        raise ValueError("a is [M x K], w is [N x K], same dtype")
+    dt = _dtype_code(a)
+    if quantize and out is None:
+        out = QBuf.empty(M * N, bits, block, a.device)
+    if not quantize:
+        out = None
+        if partial is None:
+            partial = torch.empty(M, N, dtype=a.dtype, device=a.device)
+    status = torch.zeros(4, dtype=torch.int32, device=a.device) if status is None else status
+    q = out.struct() if out is not None else None
+    _check(_lib().fc_gemm_quantize(ctypes.c_void_p(_dev_ptr(a, "a")), ctypes.c_void_p(_dev_ptr(w, "w")), dt,
+                                   M, N, K, bits, block, ctypes.byref(q) if q is not None else None,
+                                   ctypes.c_void_p(_dev_ptr(partial, "partial")) if partial is not None else None,
+                                   ctypes.c_void_p(_dev_ptr(status, "status")), _stream(stream)),
+           "fc_gemm_quantize")
+    return out, partial, status
 

@@ -3,6 +3,8 @@
 // Every entry point validates its arguments completely before it touches the
 // GPU, then launches exactly one kernel on the caller's stream and returns
 // without synchronizing.  Nothing is allocated.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <map>
@@ -10,6 +12,7 @@
 #include <utility>
 
 #include "../../include/fc.h"
+#include "fc_gemm.cuh"
 #include "fc_kernels.cuh"
 
 namespace {
@@ -316,6 +319,110 @@ fc_status fc_quantized_allreduce(const void* const* x, int P, fc_dtype dtype, si
     if (!valid_bits(bits))
         return FC_ERR_INVALID_ARG;
     return fc_quantized_allreduce_ex(x, P, dtype, n, bits, bits, block, y, step1, step2, stream);
+}
+
+}  // extern "C"
+
+namespace {
+
+// cuTensorMapEncodeTiled from the driver, fetched once through the runtime
+// (no link-time dependency on libcuda).
+PFN_cuTensorMapEncodeTiled tensor_map_encoder()
+{
+    static PFN_cuTensorMapEncodeTiled fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled>(p);
+    });
+    return fn;
+}
+
+// 2-D tensor map of a row-major [rows x K] 16-bit matrix, boxes of
+// box_rows x 64 elements (128 bytes along K) with the 128-byte swizzle.
+bool make_kmajor_map(CUtensorMap* map, const void* base, bool bf16, uint64_t rows, uint64_t K, uint32_t box_rows)
+{
+    PFN_cuTensorMapEncodeTiled enc = tensor_map_encoder();
+    if (enc == nullptr)
+        return false;
+    const cuuint64_t dims[2] = {K, rows};
+    const cuuint64_t strides[1] = {K * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)fc::GQ_BK, box_rows};
+    const cuuint32_t elem[2] = {1, 1};
+    return enc(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+               const_cast<void*>(base), dims, strides, box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+using GemmFnT = cudaError_t (*)(const CUtensorMap&, const CUtensorMap&, const fc::GemmQuantArgs&, cudaStream_t);
+// [dtype][bits == 4][log2(block) - 5]
+const GemmFnT kGemm[2][2][3] = {
+    {{fc::launch_gemm_quant<__half, 8, 32>, fc::launch_gemm_quant<__half, 8, 64>,
+      fc::launch_gemm_quant<__half, 8, 128>},
+     {fc::launch_gemm_quant<__half, 4, 32>, fc::launch_gemm_quant<__half, 4, 64>,
+      fc::launch_gemm_quant<__half, 4, 128>}},
+    {{fc::launch_gemm_quant<__nv_bfloat16, 8, 32>, fc::launch_gemm_quant<__nv_bfloat16, 8, 64>,
+      fc::launch_gemm_quant<__nv_bfloat16, 8, 128>},
+     {fc::launch_gemm_quant<__nv_bfloat16, 4, 32>, fc::launch_gemm_quant<__nv_bfloat16, 4, 64>,
+      fc::launch_gemm_quant<__nv_bfloat16, 4, 128>}},
+};
+
+}  // namespace
+
+extern "C" {
+
+fc_status fc_gemm_quantize(const void* a, const void* w, fc_dtype dtype, int M, int N, int K, int bits, int block,
+                           const fc_qbuf* out, void* partial, int* status, void* stream)
+{
+    if ((dtype != FC_FP16 && dtype != FC_BF16) || M <= 0 || N <= 0 || K <= 0 || M % fc::GQ_BM != 0 ||
+        N % fc::GQ_BN != 0 || K % fc::GQ_BK != 0 || (block != 32 && block != 64 && block != 128) ||
+        (out != nullptr && !valid_bits(bits)))
+        return FC_ERR_INVALID_ARG;
+    if (a == nullptr || w == nullptr || status == nullptr || (out == nullptr && partial == nullptr))
+        return FC_ERR_INVALID_ARG;
+    if (!aligned16(a) || !aligned16(w) || !aligned16(status) || (partial != nullptr && !aligned16(partial)))
+        return FC_ERR_MISALIGNED;
+    const size_t n = (size_t)M * (size_t)N;
+    const int qbits = out != nullptr ? bits : 8;
+    Range ins[2] = {{a, (size_t)M * (size_t)K * 2}, {w, (size_t)N * (size_t)K * 2}};
+    Range outs[5];
+    int nout = 0;
+    outs[nout++] = {status, sizeof(int)};
+    if (partial != nullptr)
+        outs[nout++] = {partial, n * 2};
+    if (out != nullptr) {
+        fc_status st = check_qbuf(out, n, qbits, block, outs + nout);
+        if (st != FC_OK)
+            return st;
+        nout += 3;
+    }
+    if (any_overlap(outs, nout, ins, 2))
+        return FC_ERR_INVALID_ARG;
+    CUtensorMap ta, tb;
+    if (!make_kmajor_map(&ta, a, dtype == FC_BF16, (uint64_t)M, (uint64_t)K, fc::GQ_BM) ||
+        !make_kmajor_map(&tb, w, dtype == FC_BF16, (uint64_t)N, (uint64_t)K, fc::GQ_BN))
+        return FC_ERR_UNSUPPORTED;
+    fc::GemmQuantArgs g{};
+    g.out = qptr(out);
+    g.partial = partial;
+    g.status = status;
+    g.M = M;
+    g.N = N;
+    g.K = K;
+    g.block = block;
+    g.tiles_m = M / fc::GQ_BM;
+    g.tiles_n = N / fc::GQ_BN;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), st);
+    if (e != cudaSuccess)
+        return cuda_fail(e);
+    const int bi = block == 32 ? 0 : block == 64 ? 1 : 2;
+    e = kGemm[dtype][qbits == 4][bi](ta, tb, g, st);
+    return e == cudaSuccess ? FC_OK : cuda_fail(e);
 }
 
 const char* fc_status_string(fc_status status)

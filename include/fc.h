@@ -142,6 +142,31 @@ fc_status fc_quantized_allreduce_ex(const void* const* x, int P, fc_dtype dtype,
                                     int bits_ag, int block, void* y, const fc_qbuf* step1,
                                     const fc_qbuf* step2, void* stream);
 
+/* One rank's tensor-parallel partial GEMM with the step-1 quantizer fused into
+ * its epilogue (page: Fig. 3, the tensor-parallel block whose attention output
+ * projection and MLP down projection produce the partial sums; Fig. 5 left,
+ * the all-reduce after each of them).
+ *   a       device, [M x K] row-major fp16/bf16 (the rank's activations);
+ *   w       device, [N x K] row-major fp16/bf16 (the rank's weight slice, in
+ *           the usual [out_features x in_features] layout);
+ *   partial = a * w^T with fp32 accumulation on the tensor cores, each value
+ *           rounded (nearest even) to dtype.  The summation order inside the
+ *           tensor cores is the hardware's, so the partial matches an exact
+ *           product to within fp32 accumulation error, not bit for bit.
+ *   out     when non-NULL: the step-1 payload of the [M x N] partial at
+ *           `bits`, blocks of `block` along N -- bit-identical to calling
+ *           fc_quantize on the partial;
+ *   partial when non-NULL: receives the [M x N] partial itself.
+ *   status  device int, required: set to 0 on the stream before the kernel and
+ *           OR-ed with 1 if a pipeline wait inside the kernel gave up (the
+ *           kernel then stops early instead of hanging; outputs are invalid).
+ * At least one of out / partial must be non-NULL.  Requires M % 128 == 0,
+ * N % 256 == 0, K % 64 == 0, block in {32, 64, 128}, bits in {4, 8}; 16-byte
+ * aligned pointers; outputs must not overlap a or w.  Each call runs one
+ * persistent kernel (one CTA per SM, 197 KB shared memory, 512 TMEM columns). */
+fc_status fc_gemm_quantize(const void* a, const void* w, fc_dtype dtype, int M, int N, int K, int bits, int block,
+                           const fc_qbuf* out, void* partial, int* status, void* stream);
+
 /* Static description of a status code. */
 const char* fc_status_string(fc_status status);
 
