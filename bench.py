@@ -265,6 +265,64 @@ def run_precision_sweep(args, w):
             del s1, s2
 
 
+def run_gemm(args):
+    """The GEMM with the fused step-1 quantizer (tensor cores), on the o_proj
+    shape of the 70B-shaped workload: one rank's partial of [8192 tokens x 8192
+    hidden] over its K = 8192/4 = 2048 slice, INT8 blocks of 128.  Compared
+    with cuBLAS for the same GEMM followed by the separate quantize kernel."""
+    import torch
+
+    import bit_quantized_all_block_b200 as fc
+
+    torch.cuda.set_device(0)
+    M, N, K = args.gemm_shape
+    g = torch.Generator().manual_seed(0)
+    a = torch.randn(M, K, generator=g).bfloat16().cuda()
+    w = (torch.randn(N, K, generator=g) / K ** 0.5).bfloat16().cuda()
+    q = fc.QBuf.empty(M * N, 8, 128)
+    part = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    status = torch.zeros(4, dtype=torch.int32, device="cuda")
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.steps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / args.steps
+
+    with ClockSampler(0) as clocks:
+        ms_fused = timed(lambda: fc.fc_gemm_quantize(a, w, 8, 128, out=q, status=status))
+    assert int(status[0].item()) == 0, "GEMM pipeline reported a timeout"
+    ms_plain = timed(lambda: fc.fc_gemm_quantize(a, w, 8, 128, partial=part, status=status, quantize=False))
+    ms_cublas = timed(lambda: torch.matmul(a, w.t(), out=part))
+    ms_quant = timed(lambda: fc.fc_quantize(part.view(-1), 8, 128, out=q))
+    flops = 2.0 * M * N * K
+    tflops = flops / (ms_fused * 1e-3) / 1e12
+    try:
+        d = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+        peak, kind = float(d["bf16_tflops"]), "measured burst"
+    except (OSError, KeyError, ValueError):
+        peak, kind = 1590.0, "fallback"
+    print(json.dumps({
+        "metric": "GEMM with fused step-1 quantization, TFLOP/s", "mode": "gemm", "value": round(tflops, 1),
+        "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "us_per_call": round(ms_fused * 1e3, 2), "higher_is_better": True, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": f"o_proj partial per rank M={M} N={N} K={K}, bf16, INT8 block 128"},
+        "roofline": {"bound": "tensor", "achieved": round(tflops, 1), "peak": peak, "unit": "TFLOP/s",
+                     "frac": round(tflops / peak, 4), "peak_kind": kind},
+        "compare_us": {"fused_gemm_quantize": round(ms_fused * 1e3, 2),
+                       "our_gemm_partial_only": round(ms_plain * 1e3, 2),
+                       "cublas_gemm": round(ms_cublas * 1e3, 2), "quantize_kernel": round(ms_quant * 1e3, 2),
+                       "cublas_gemm_then_quantize": round((ms_cublas + ms_quant) * 1e3, 2)},
+        "gpu_launches": args.steps, "clocks": clocks.summary()}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -282,6 +340,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch the timed steps one by one instead of replaying a CUDA graph of them")
+    ap.add_argument("--gemm", action="store_true",
+                    help="time the tensor-core GEMM with the fused step-1 quantizer (o_proj shape)")
+    ap.add_argument("--gemm-shape", type=int, nargs=3, default=[8192, 8192, 2048], metavar=("M", "N", "K"))
     ap.add_argument("--precision-sweep", action="store_true",
                     help="time the fused kernel for every (RS bits, AG bits) in {4,8,16}^2 on the "
                          "workload and report each variant's MSE (one JSON line per variant)")
@@ -294,6 +355,8 @@ def main():
         return run_reference(args, w)
     if args.precision_sweep:
         return run_precision_sweep(args, w)
+    if args.gemm:
+        return run_gemm(args)
 
     import torch
     import torch.distributed as dist
