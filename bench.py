@@ -48,7 +48,9 @@ METRIC = "quantized all-reduce input GB/s and % of HBM roofline (1×B200)"
 FALLBACK_HBM_GBS = 6650.0
 L2_FLUSH_THRESHOLD = 256 << 20     # steps moving less than ~2x L2 (126 MB) get a cold-L2 timing
 FLUSH_BYTES = 512 << 20
-KERNEL_SOURCES = sorted(glob.glob(os.path.join(ROOT, "bit_quantized_all_block_b200", "csrc", "*.cu*")))
+# sources of the fused all-reduce kernel (the dominant kernel of the default bench)
+KERNEL_SOURCES = [os.path.join(ROOT, "bit_quantized_all_block_b200", "csrc", f)
+                  for f in ("fc_device.cuh", "fc_kernels.cuh", "fc_fused.cuh", "fc_launch_impl.cuh")]
 
 
 def payload_bytes(w) -> int:
