@@ -124,6 +124,28 @@ const FusedFnT kFused[2][3][3][8] = {FC_DTYPE(__half), FC_DTYPE(__nv_bfloat16)};
 
 int width_index(int bits) { return bits == 4 ? 0 : bits == 8 ? 1 : bits == 16 ? 2 : -1; }
 
+// The fused kernel's latency shape (64-thread CTAs, 8 elements per thread) for
+// decode-sized messages: equal quantized widths, P in {2, 4, 8}, blocks of at
+// most 256, and at most FC_SMALL_MAX_ELEMS elements over all ranks.
+#ifndef FC_SMALL_MAX_ELEMS
+#define FC_SMALL_MAX_ELEMS (1u << 20)
+#endif
+#define FC_SMALL(T, B) {fc::launch_fused<T, B, B, 2, true>, fc::launch_fused<T, B, B, 4, true>, fc::launch_fused<T, B, B, 8, true>}
+// [dtype][bits == 4][P = 2, 4, 8]
+const FusedFnT kFusedSmall[2][2][3] = {
+    {FC_SMALL(__half, 8), FC_SMALL(__half, 4)},
+    {FC_SMALL(__nv_bfloat16, 8), FC_SMALL(__nv_bfloat16, 4)},
+};
+#undef FC_SMALL
+
+FusedFnT small_variant(fc_dtype dtype, int bits_rs, int bits_ag, int P, int block, size_t n)
+{
+    if (bits_rs != bits_ag || bits_rs == 16 || block > 256 || n * (size_t)P > (size_t)FC_SMALL_MAX_ELEMS)
+        return nullptr;
+    const int pi = P == 2 ? 0 : P == 4 ? 1 : P == 8 ? 2 : -1;
+    return pi < 0 ? nullptr : kFusedSmall[dtype][bits_rs == 4][pi];
+}
+
 }  // namespace
 
 namespace fc {
@@ -262,9 +284,11 @@ fc_status fc_quantized_allreduce_ex(const void* const* x, int P, fc_dtype dtype,
         return FC_ERR_INVALID_ARG;
     if ((bits_rs == 16 && step1 != nullptr) || (bits_ag == 16 && step2 != nullptr))
         return FC_ERR_INVALID_ARG;   // an unquantized step has no payload
-    const FusedFnT fn = kFused[dtype][w1][w2][P - 1];
+    FusedFnT fn = kFused[dtype][w1][w2][P - 1];
     if (fn == nullptr)
         return FC_ERR_UNSUPPORTED;
+    if (FusedFnT small = small_variant(dtype, bits_rs, bits_ag, P, block, n))
+        fn = small;
     if (n == 0)
         return FC_OK;
     if (x == nullptr || y == nullptr)

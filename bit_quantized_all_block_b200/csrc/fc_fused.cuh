@@ -42,11 +42,19 @@ constexpr int FU_THREADS = 256;
 #define FC_FUSED_MIN_CTAS 2
 #endif
 
-template <int P>
+// Launch shape.  The bandwidth shape (SMALL = false): 256-thread CTAs, two CTAs
+// per SM, 16 elements per thread per rank.  The latency shape for
+// decode-sized messages (SMALL = true): 64-thread CTAs with 8 elements per
+// thread per rank, so a call of a few hundred KB spreads over many more SMs
+// and each thread's dependent chain is half as long; it serves blocks of up to
+// 256 elements (a block must fit in one warp: 32 threads x 8).
+template <int P, bool SMALL = false>
 struct FuShape {
-    static constexpr int NC = P <= 4 ? FC_FUSED_NC_SMALL_P : 2;   // 16-byte chunks per thread per rank
+    static constexpr int THREADS = SMALL ? 64 : FU_THREADS;
+    static constexpr int NC = SMALL ? 1 : (P <= 4 ? FC_FUSED_NC_SMALL_P : 2);  // 16-byte chunks per thread per rank
     static constexpr int E = NC * FC_CHUNK;                       // elements per thread per rank
-    static constexpr int TILE = FU_THREADS * E;                   // elements per rank per tile
+    static constexpr int TILE = THREADS * E;                      // elements per rank per tile
+    static constexpr int MIN_CTAS = SMALL ? 8 : FC_FUSED_MIN_CTAS;
 };
 
 __device__ __forceinline__ uint4 ld_nc(const void* p)
@@ -121,8 +129,10 @@ __device__ __forceinline__ void store_thread_codes(uint8_t* codes, size_t e, con
 #pragma unroll
         for (int i = 0; i < NW; i += 4)
             st_stream(p + 4 * i, make_uint4(w[i], w[i + 1], w[i + 2], w[i + 3]));
-    } else {
+    } else if constexpr (NW == 2) {
         st_stream(p, make_uint2(w[0], w[1]));
+    } else {
+        st_stream(p, w[0]);
     }
 }
 
@@ -247,15 +257,17 @@ __device__ __forceinline__ void rank_body_plain(const uint4* raw, float* acc)
 // B1 / B2: bits of the reduce-scatter and of the all-gather step, each 4, 8
 // or 16 (16 = that step sends fp16/bf16 values unquantized; Fig. 5 right of
 // the page compares quantizing before RS with quantizing before AG).
-template <class T, int B1, int B2, int P>
-__global__ void __launch_bounds__(FU_THREADS, FC_FUSED_MIN_CTAS) k_fused(const FusedArgs a)
+template <class T, int B1, int B2, int P, bool SMALL = false>
+__global__ void __launch_bounds__(FuShape<P, SMALL>::THREADS, FuShape<P, SMALL>::MIN_CTAS)
+    k_fused(const FusedArgs a)
 {
     using P2 = Pair<T>;
     using T2 = typename P2::T2;
-    constexpr int NC = FuShape<P>::NC, E = FuShape<P>::E, TILE = FuShape<P>::TILE;
+    using S = FuShape<P, SMALL>;
+    constexpr int NC = S::NC, E = S::E, TILE = S::TILE;
     constexpr int QB1 = B1 == 16 ? 8 : B1;     // (unused when B1 == 16)
-    __shared__ uint32_t red16[P][FU_THREADS / 32];
-    __shared__ float2 red32[FU_THREADS / 32];
+    __shared__ uint32_t red16[P][S::THREADS / 32];
+    __shared__ float2 red32[S::THREADS / 32];
 
     const int L = a.block / E;                 // threads per block (1 .. 256)
     const int j = threadIdx.x % L;             // member index inside the block

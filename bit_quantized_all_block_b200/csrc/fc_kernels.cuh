@@ -61,7 +61,8 @@ struct FusedArgs {
 template <class T, int BITS> cudaError_t launch_quantize(const QuantArgs& a, cudaStream_t st);
 template <int BITS, int P> cudaError_t launch_rs(const RsArgs& a, cudaStream_t st);
 template <class T, int BITS> cudaError_t launch_ag(const AgArgs& a, cudaStream_t st);
-template <class T, int B1, int B2, int P> cudaError_t launch_fused(const FusedArgs& a, cudaStream_t st);
+template <class T, int B1, int B2, int P, bool SMALL = false>
+cudaError_t launch_fused(const FusedArgs& a, cudaStream_t st);
 
 // Persistent grid: enough CTAs of `threads` threads to fill every SM at the
 // kernel's occupancy, never more than there are tiles of `tile` elements.

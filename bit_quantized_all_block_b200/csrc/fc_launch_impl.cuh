@@ -38,14 +38,15 @@ cudaError_t launch_ag(const AgArgs& a, cudaStream_t st)
     return cudaGetLastError();
 }
 
-template <class T, int B1, int B2, int P>
+template <class T, int B1, int B2, int P, bool SMALL>
 cudaError_t launch_fused(const FusedArgs& a, cudaStream_t st)
 {
+    using S = FuShape<P, SMALL>;
     int grid = 0;
-    cudaError_t e = persistent_grid((const void*)k_fused<T, B1, B2, P>, FU_THREADS, a.n, FuShape<P>::TILE, &grid);
+    cudaError_t e = persistent_grid((const void*)k_fused<T, B1, B2, P, SMALL>, S::THREADS, a.n, S::TILE, &grid);
     if (e != cudaSuccess)
         return e;
-    k_fused<T, B1, B2, P><<<grid, FU_THREADS, 0, st>>>(a);
+    k_fused<T, B1, B2, P, SMALL><<<grid, S::THREADS, 0, st>>>(a);
     return cudaGetLastError();
 }
 
