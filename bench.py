@@ -325,6 +325,58 @@ def run_gemm(args):
         "gpu_launches": args.steps, "clocks": clocks.summary()}), flush=True)
 
 
+def run_latency_sweep(args):
+    """Decode regime: per-call latency of the fused all-reduce over the message
+    sweep (16 KB .. 8 MB per rank, P=4, INT8 and INT4), measured two ways:
+    back to back inside a CUDA graph (L2 warm: the kernel's own latency) and
+    one call at a time after an L2 flush (cold)."""
+    import torch
+
+    import bit_quantized_all_block_b200 as fc
+
+    torch.cuda.set_device(0)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    for bits in (8, 4):
+        for w in synth.message_sweep(bits)[:10]:
+            xs = [torch.from_numpy(x.view(np.int16)).view(torch.float16).cuda() for x in synth.workload_partials(w)]
+            y = torch.empty(w.n, dtype=torch.float16, device="cuda")
+            s1 = [fc.QBuf.empty(w.n, bits, w.block) for _ in range(w.P)]
+            s2 = fc.QBuf.empty(w.n, bits, w.block)
+
+            def step():
+                fc.fc_quantized_allreduce(xs, bits, w.block, y=y, step1=s1, step2=s2)
+
+            for _ in range(args.warmup):
+                step()
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                for _ in range(20):
+                    step()
+            g.replay()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            g.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            hot = e0.elapsed_time(e1) * 1e3 / 20
+            pairs = []
+            for _ in range(args.steps):
+                flush.zero_()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record()
+                step()
+                b.record()
+                pairs.append((a, b))
+            torch.cuda.synchronize()
+            cold = sorted(a.elapsed_time(b) * 1e3 for a, b in pairs)[len(pairs) // 2]
+            print(json.dumps({"mode": "latency_sweep", "workload": w.name, "bytes_per_rank": 2 * w.n,
+                              "us_graph_back_to_back": round(hot, 2), "us_cold_l2_median": round(cold, 2),
+                              "input_gbs_back_to_back": round(w.P * w.n * 2 / hot / 1e3, 1)}), flush=True)
+            del g
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -345,6 +397,8 @@ def main():
     ap.add_argument("--gemm", action="store_true",
                     help="time the tensor-core GEMM with the fused step-1 quantizer (o_proj shape)")
     ap.add_argument("--gemm-shape", type=int, nargs=3, default=[8192, 8192, 2048], metavar=("M", "N", "K"))
+    ap.add_argument("--latency-sweep", action="store_true",
+                    help="decode regime: per-call latency over the 16 KB .. 8 MB per rank message sweep")
     ap.add_argument("--precision-sweep", action="store_true",
                     help="time the fused kernel for every (RS bits, AG bits) in {4,8,16}^2 on the "
                          "workload and report each variant's MSE (one JSON line per variant)")
@@ -359,6 +413,8 @@ def main():
         return run_precision_sweep(args, w)
     if args.gemm:
         return run_gemm(args)
+    if args.latency_sweep:
+        return run_latency_sweep(args)
 
     import torch
     import torch.distributed as dist
