@@ -22,7 +22,7 @@
 //  * the upper code clamp binds only when the block maximum's code rounds to
 //    qmax + 1 -- rare -- so it is checked once per block from the maximum and
 //    applied through a warp-uniform branch; the lower clamp never binds
-//    (see quant_shifted in fc_device.cuh);
+//    (see the lower-clamp note in fc_device.cuh);
 //  * each rank's registers are refilled with the next tile's data as soon as
 //    that rank is consumed, so loads stay in flight during the rest of the
 //    tile (software pipelining without extra registers);
