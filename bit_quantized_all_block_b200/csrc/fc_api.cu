@@ -394,6 +394,20 @@ const GemmFnT kGemm[2][2][3] = {
      {fc::launch_gemm_quant<__nv_bfloat16, 4, 32>, fc::launch_gemm_quant<__nv_bfloat16, 4, 64>,
       fc::launch_gemm_quant<__nv_bfloat16, 4, 128>}},
 };
+// The SM-pair kernel (256 x 256 tiles), used when M is a multiple of 256.
+const GemmFnT kGemmPair[2][2][3] = {
+    {{fc::launch_gemm_quant_pair<__half, 8, 32>, fc::launch_gemm_quant_pair<__half, 8, 64>,
+      fc::launch_gemm_quant_pair<__half, 8, 128>},
+     {fc::launch_gemm_quant_pair<__half, 4, 32>, fc::launch_gemm_quant_pair<__half, 4, 64>,
+      fc::launch_gemm_quant_pair<__half, 4, 128>}},
+    {{fc::launch_gemm_quant_pair<__nv_bfloat16, 8, 32>, fc::launch_gemm_quant_pair<__nv_bfloat16, 8, 64>,
+      fc::launch_gemm_quant_pair<__nv_bfloat16, 8, 128>},
+     {fc::launch_gemm_quant_pair<__nv_bfloat16, 4, 32>, fc::launch_gemm_quant_pair<__nv_bfloat16, 4, 64>,
+      fc::launch_gemm_quant_pair<__nv_bfloat16, 4, 128>}},
+};
+#ifndef FC_GEMM_PAIR
+#define FC_GEMM_PAIR 1
+#endif
 
 }  // namespace
 
@@ -426,9 +440,10 @@ fc_status fc_gemm_quantize(const void* a, const void* w, fc_dtype dtype, int M, 
     }
     if (any_overlap(outs, nout, ins, 2))
         return FC_ERR_INVALID_ARG;
+    const bool pair = FC_GEMM_PAIR && M % 256 == 0;   // SM pairs: each CTA loads 128 rows of W
     CUtensorMap ta, tb;
     if (!make_kmajor_map(&ta, a, dtype == FC_BF16, (uint64_t)M, (uint64_t)K, fc::GQ_BM) ||
-        !make_kmajor_map(&tb, w, dtype == FC_BF16, (uint64_t)N, (uint64_t)K, fc::GQ_BN))
+        !make_kmajor_map(&tb, w, dtype == FC_BF16, (uint64_t)N, (uint64_t)K, pair ? 128 : fc::GQ_BN))
         return FC_ERR_UNSUPPORTED;
     fc::GemmQuantArgs g{};
     g.out = qptr(out);
@@ -445,7 +460,7 @@ fc_status fc_gemm_quantize(const void* a, const void* w, fc_dtype dtype, int M, 
     if (e != cudaSuccess)
         return cuda_fail(e);
     const int bi = block == 32 ? 0 : block == 64 ? 1 : 2;
-    e = kGemm[dtype][qbits == 4][bi](ta, tb, g, st);
+    e = (pair ? kGemmPair : kGemm)[dtype][qbits == 4][bi](ta, tb, g, st);
     return e == cudaSuccess ? FC_OK : cuda_fail(e);
 }
 

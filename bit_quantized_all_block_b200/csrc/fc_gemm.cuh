@@ -415,4 +415,247 @@ template <class T, int BITS, int NB>
 cudaError_t launch_gemm_quant(const CUtensorMap& ta, const CUtensorMap& tb, const GemmQuantArgs& a,
                               cudaStream_t st);
 
+
+// ============================================================================
+// The same GEMM on SM pairs: a cluster of two CTAs computes a 256 x 256 tile
+// with tcgen05.mma.cta_group::2 (M = 256 across the pair, N = 256).  Each CTA
+// loads its own 128-row halves of the A tile and of the W tile, so each SM
+// reads half the W traffic of the one-SM kernel from L2 and a stage is 32 KB,
+// which leaves room for 6 stages.  The leader CTA (cluster rank 0) issues the
+// MMAs; the loads of both CTAs complete on the leader's stage barrier, the
+// leader's commits are multicast to the matching barriers of both CTAs, and
+// the epilogue warps of both CTAs arrive on the leader's accumulator barrier.
+// Loads carry no multicast: every CTA fetches its own operands.
+// ============================================================================
+constexpr int G2_STAGES = 6;
+constexpr int G2_A_BYTES = 128 * GQ_BK * 2;     // 16 KB: this CTA's 128 rows of A
+constexpr int G2_B_BYTES = 128 * GQ_BK * 2;     // 16 KB: this CTA's 128 rows of W (half of N)
+constexpr int G2_STAGE_BYTES = G2_A_BYTES + G2_B_BYTES;
+constexpr int G2_SMEM_BYTES = G2_STAGES * G2_STAGE_BYTES + 1024 + 256;
+
+__device__ __forceinline__ uint32_t cluster_rank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ void cluster_sync_all()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Arrive on the barrier at the same shared-memory offset in CTA `rank` of the cluster.
+__device__ __forceinline__ void mbar_arrive_cluster(uint64_t* bar, uint32_t rank)
+{
+    uint32_t remote;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(bar)), "r"(rank));
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote) : "memory");
+}
+
+// TMA load into this CTA's shared memory whose completion is counted on the
+// pair leader's barrier (the barrier at the same offset in CTA rank 0, as a
+// shared::cluster address).
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y)
+{
+    uint32_t leader_bar;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, 0;" : "=r"(leader_bar) : "r"(smem_u32(bar)));
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];"
+        ::"r"(smem_u32(dst)), "l"(map), "r"(leader_bar), "r"(x), "r"(y)
+        : "memory");
+}
+
+__device__ __forceinline__ void umma_f16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                              uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n"
+        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+
+// Commit: arrive on the barrier at this offset in both CTAs of the pair once
+// every MMA issued so far has completed.
+__device__ __forceinline__ void umma_commit_pair(uint64_t* bar)
+{
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
+        ::"r"(smem_u32(bar)), "h"((uint16_t)0x3) : "memory");
+}
+
+template <class T>
+__host__ __device__ constexpr uint32_t umma_idesc_256x256()
+{
+    constexpr uint32_t ab = std::is_same<T, __nv_bfloat16>::value ? 1u : 0u;
+    return (1u << 4) | (ab << 7) | (ab << 10) | ((uint32_t)(256 >> 3) << 17) | ((uint32_t)(256 >> 4) << 24);
+}
+
+template <class T, int BITS, int NB>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GQ_THREADS, 1)
+    k_gemm_quant_pair(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                      const GemmQuantArgs a)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sA = smem;
+    uint8_t* sB = smem + G2_STAGES * G2_A_BYTES;
+    uint64_t* full = reinterpret_cast<uint64_t*>(sB + G2_STAGES * G2_B_BYTES);
+    uint64_t* empty = full + G2_STAGES;
+    uint64_t* acc_full = empty + G2_STAGES;      // [2]
+    uint64_t* acc_empty = acc_full + 2;          // [2] (the leader's is used)
+    uint64_t* drain = acc_empty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t crank = cluster_rank();
+    const bool leader = crank == 0;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < G2_STAGES; s++) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; b++) {
+            mbar_init(&acc_full[b], 1);
+            mbar_init(&acc_empty[b], 8);     // four epilogue warps in each CTA of the pair
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;"
+                     ::"r"(smem_u32(tmem_slot)), "r"(GQ_TMEM_COLS));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    cluster_sync_all();          // both CTAs' barriers initialised before any remote use
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const int tiles_m2 = a.tiles_m / 2;          // 256-row tiles
+    const int num_tiles = tiles_m2 * a.tiles_n;
+    const int kblocks = a.K / GQ_BK;
+    const int cluster_id = blockIdx.x >> 1, num_clusters = gridDim.x >> 1;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---- TMA producer (both CTAs) ----
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t issued = 0, issued_parity = 0;
+            bool ok = true;
+            for (int tile = cluster_id; tile < num_tiles && ok; tile += num_clusters) {
+                const int m2 = tile % tiles_m2, n_blk = tile / tiles_m2;
+                const int a_row = m2 * 256 + 128 * (int)crank, b_row = n_blk * GQ_BN + 128 * (int)crank;
+                for (int kb = 0; kb < kblocks; kb++) {
+                    if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    if (leader)
+                        mbar_expect_tx(&full[stage], 2 * G2_STAGE_BYTES);
+                    tma_load_2d_pair(sA + stage * G2_A_BYTES, &tmap_a, &full[stage], kb * GQ_BK, a_row);
+                    tma_load_2d_pair(sB + stage * G2_B_BYTES, &tmap_b, &full[stage], kb * GQ_BK, b_row);
+                    issued |= 1u << stage;
+                    issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+                    if (++stage == G2_STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (!ok && leader) {   // the leader's stage barriers count both CTAs' loads
+                for (int s = 0; s < G2_STAGES; s++)
+                    if (issued & (1u << s))
+                        wait_drain(&full[s], (issued_parity >> s) & 1u);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && leader) {
+            // ---- MMA issuer (leader CTA) ----
+            constexpr uint32_t idesc = umma_idesc_256x256<T>();
+            int stage = 0, acc = 0;
+            uint32_t phase = 0, acc_phase = 0;
+            bool ok = true, any = false;
+            for (int tile = cluster_id; tile < num_tiles && ok; tile += num_clusters) {
+                if (!wait_bounded(&acc_empty[acc], acc_phase ^ 1u, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * GQ_BN);
+                for (int kb = 0; kb < kblocks; kb++) {
+                    if (!wait_bounded(&full[stage], phase, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t ad = smem_desc_k_sw128(sA + stage * G2_A_BYTES);
+                    const uint64_t bd = smem_desc_k_sw128(sB + stage * G2_B_BYTES);
+#pragma unroll
+                    for (int k = 0; k < GQ_BK / 16; k++)
+                        umma_f16_pair(d_tmem, ad + 2 * k, bd + 2 * k, idesc, (kb | k) != 0);
+                    any = true;
+                    umma_commit_pair(&empty[stage]);
+                    if (++stage == G2_STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok)
+                    break;
+                umma_commit_pair(&acc_full[acc]);
+                acc ^= 1;
+                if (acc == 0)
+                    acc_phase ^= 1u;
+            }
+            if (!ok && any) {
+                umma_commit_pair(drain);
+                wait_drain(drain, 0);
+            }
+        }
+    } else {
+        // ---- epilogue: warps 2..5 of both CTAs ----
+        const int quad = warp & 3;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int tile = cluster_id; tile < num_tiles; tile += num_clusters) {
+            const int m2 = tile % tiles_m2, n_blk = tile / tiles_m2;
+            if (!wait_bounded(&acc_full[acc], acc_phase, abort_flag))
+                break;
+            tc_fence_after();
+            const uint32_t taddr = tmem_base + ((uint32_t)(32 * quad) << 16) + (uint32_t)(acc * GQ_BN);
+            const size_t row = (size_t)m2 * 256 + 128 * crank + 32 * quad + lane;
+#pragma unroll 1
+            for (int c = 0; c < GQ_BN; c += NB)
+                epilogue_block<T, BITS, NB>(taddr + c, a, row, n_blk * GQ_BN + c);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive_cluster(&acc_empty[acc], 0);
+            acc ^= 1;
+            if (acc == 0)
+                acc_phase ^= 1u;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync_all();          // neither CTA leaves while the pair's MMAs or barriers are in use
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(GQ_TMEM_COLS)
+                     : "memory");
+    }
+    if (threadIdx.x == 0 && *abort_flag)
+        atomicOr(a.status, GQ_STATUS_TIMEOUT);
+}
+
+template <class T, int BITS, int NB>
+cudaError_t launch_gemm_quant_pair(const CUtensorMap& ta, const CUtensorMap& tb, const GemmQuantArgs& a,
+                                   cudaStream_t st);
+
 }  // namespace fc

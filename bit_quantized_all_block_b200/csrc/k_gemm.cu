@@ -42,6 +42,39 @@ cudaError_t launch_gemm_quant(const CUtensorMap& ta, const CUtensorMap& tb, cons
     return cudaGetLastError();
 }
 
+template <class T, int BITS, int NB>
+cudaError_t launch_gemm_quant_pair(const CUtensorMap& ta, const CUtensorMap& tb, const GemmQuantArgs& a,
+                                   cudaStream_t st)
+{
+    static std::mutex mu;
+    static std::map<int, int> sms_of;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return e;
+    int sms = 0;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        auto it = sms_of.find(dev);
+        if (it == sms_of.end()) {
+            e = cudaFuncSetAttribute(k_gemm_quant_pair<T, BITS, NB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     G2_SMEM_BYTES);
+            if (e != cudaSuccess)
+                return e;
+            e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+            if (e != cudaSuccess)
+                return e;
+            sms_of[dev] = sms;
+        } else {
+            sms = it->second;
+        }
+    }
+    const int pairs_needed = (a.tiles_m / 2) * a.tiles_n;
+    const int pairs = pairs_needed < sms / 2 ? pairs_needed : sms / 2;
+    k_gemm_quant_pair<T, BITS, NB><<<2 * pairs, GQ_THREADS, G2_SMEM_BYTES, st>>>(ta, tb, a);
+    return cudaGetLastError();
+}
+
 #define FC_GQ(T)                                                                                  \
     template cudaError_t launch_gemm_quant<T, 8, 32>(const CUtensorMap&, const CUtensorMap&,      \
                                                      const GemmQuantArgs&, cudaStream_t);         \
@@ -58,5 +91,14 @@ cudaError_t launch_gemm_quant(const CUtensorMap& ta, const CUtensorMap& tb, cons
 FC_GQ(__half)
 FC_GQ(__nv_bfloat16)
 #undef FC_GQ
+
+#define FC_GQ2(T, B, NB)                                                                           \
+    template cudaError_t launch_gemm_quant_pair<T, B, NB>(const CUtensorMap&, const CUtensorMap&,  \
+                                                          const GemmQuantArgs&, cudaStream_t);
+FC_GQ2(__half, 8, 32) FC_GQ2(__half, 8, 64) FC_GQ2(__half, 8, 128)
+FC_GQ2(__half, 4, 32) FC_GQ2(__half, 4, 64) FC_GQ2(__half, 4, 128)
+FC_GQ2(__nv_bfloat16, 8, 32) FC_GQ2(__nv_bfloat16, 8, 64) FC_GQ2(__nv_bfloat16, 8, 128)
+FC_GQ2(__nv_bfloat16, 4, 32) FC_GQ2(__nv_bfloat16, 4, 64) FC_GQ2(__nv_bfloat16, 4, 128)
+#undef FC_GQ2
 
 }  // namespace fc
