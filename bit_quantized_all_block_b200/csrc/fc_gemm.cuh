@@ -196,6 +196,23 @@ __device__ __forceinline__ void tmem_ld_32cols(uint32_t taddr, uint32_t* r)
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// Tile order: groups of GQ_GROUP_M row blocks, all column blocks of a group
+// before the next group, row blocks fastest inside a group.  The tiles that
+// run at the same time then share a few row blocks of A and column blocks of
+// W, so both stay in L2 even when the operands together exceed it.
+constexpr int GQ_GROUP_M = 8;
+
+__device__ __forceinline__ void tile_coords(int tile, int tiles_m, int tiles_n, int& m, int& n)
+{
+    const int per_group = GQ_GROUP_M * tiles_n;
+    const int g = tile / per_group;
+    const int first_m = g * GQ_GROUP_M;
+    const int gsize = min(GQ_GROUP_M, tiles_m - first_m);
+    const int r = tile - g * per_group;
+    m = first_m + r % gsize;
+    n = r / gsize;
+}
+
 // ---- epilogue: one row's block of `NB` columns ---------------------------------
 // The 16-bit partial values of the block (rounded from fp32, nearest even)
 // are kept as packed pairs; the block is quantized exactly as fc_quantize
@@ -306,7 +323,8 @@ __global__ void __launch_bounds__(GQ_THREADS, 1)
             uint32_t issued_parity = 0;     // bit s: parity of that load's phase
             bool ok = true;
             for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-                const int m_blk = tile % a.tiles_m, n_blk = tile / a.tiles_m;
+                int m_blk, n_blk;
+                tile_coords(tile, a.tiles_m, a.tiles_n, m_blk, n_blk);
                 for (int kb = 0; kb < kblocks; kb++) {
                     if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag)) {
                         ok = false;
@@ -380,7 +398,8 @@ __global__ void __launch_bounds__(GQ_THREADS, 1)
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-            const int m_blk = tile % a.tiles_m, n_blk = tile / a.tiles_m;
+            int m_blk, n_blk;
+            tile_coords(tile, a.tiles_m, a.tiles_n, m_blk, n_blk);
             if (!wait_bounded(&acc_full[acc], acc_phase, abort_flag))
                 break;
             tc_fence_after();
@@ -547,7 +566,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GQ_THREADS, 1)
             uint32_t issued = 0, issued_parity = 0;
             bool ok = true;
             for (int tile = cluster_id; tile < num_tiles && ok; tile += num_clusters) {
-                const int m2 = tile % tiles_m2, n_blk = tile / tiles_m2;
+                int m2, n_blk;
+                tile_coords(tile, tiles_m2, a.tiles_n, m2, n_blk);
                 const int a_row = m2 * 256 + 128 * (int)crank, b_row = n_blk * GQ_BN + 128 * (int)crank;
                 for (int kb = 0; kb < kblocks; kb++) {
                     if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag)) {
@@ -622,7 +642,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GQ_THREADS, 1)
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int tile = cluster_id; tile < num_tiles; tile += num_clusters) {
-            const int m2 = tile % tiles_m2, n_blk = tile / tiles_m2;
+            int m2, n_blk;
+            tile_coords(tile, tiles_m2, a.tiles_n, m2, n_blk);
             if (!wait_bounded(&acc_full[acc], acc_phase, abort_flag))
                 break;
             tc_fence_after();
