@@ -303,6 +303,30 @@ def run_gemm(args):
     ms_plain = timed(lambda: fc.fc_gemm_quantize(a, w, 8, 128, partial=part, status=status, quantize=False))
     ms_cublas = timed(lambda: torch.matmul(a, w.t(), out=part))
     ms_quant = timed(lambda: fc.fc_quantize(part.view(-1), 8, 128, out=q))
+    # The whole tensor-parallel layer output for P ranks (the page's setting:
+    # each rank's o_proj partial, then the all-reduce), three ways.
+    P = args.gemm_ranks
+    As = [torch.randn(M, K, generator=g).bfloat16().cuda() for _ in range(P)]
+    Ws = [(torch.randn(N, K, generator=g) / K ** 0.5).bfloat16().cuda() for _ in range(P)]
+    q1 = [fc.QBuf.empty(M * N, 8, 128) for _ in range(P)]
+    q2 = fc.QBuf.empty(M * N, 8, 128)
+    parts = [torch.empty(M, N, dtype=torch.bfloat16, device="cuda") for _ in range(P)]
+    yb = torch.empty(M * N, dtype=torch.bfloat16, device="cuda")
+
+    def layer_fused():
+        for r in range(P):
+            fc.fc_gemm_quantize(As[r], Ws[r], 8, 128, out=q1[r], status=status)
+        fc.fc_rs_dequant_sum_requant(q1, 8, 128, out=q2)
+        fc.fc_ag_dequant(q2, torch.bfloat16, y=yb)
+
+    def layer_unfused(b):
+        for r in range(P):
+            torch.matmul(As[r], Ws[r].t(), out=parts[r])
+        fc.fc_quantized_allreduce_ex([p_.view(-1) for p_ in parts], b, b, 128, y=yb)
+
+    ms_layer_fused = timed(layer_fused)
+    ms_layer_cublas_q8 = timed(lambda: layer_unfused(8))
+    ms_layer_cublas_16 = timed(lambda: layer_unfused(16))
     flops = 2.0 * M * N * K
     tflops = flops / (ms_fused * 1e-3) / 1e12
     try:
@@ -322,6 +346,10 @@ def run_gemm(args):
                        "our_gemm_partial_only": round(ms_plain * 1e3, 2),
                        "cublas_gemm": round(ms_cublas * 1e3, 2), "quantize_kernel": round(ms_quant * 1e3, 2),
                        "cublas_gemm_then_quantize": round((ms_cublas + ms_quant) * 1e3, 2)},
+        "tp_layer_us": {"ranks": P,
+                        "fused_gemm_quantize_then_rs_ag_int8": round(ms_layer_fused * 1e3, 2),
+                        "cublas_gemms_then_fused_allreduce_int8": round(ms_layer_cublas_q8 * 1e3, 2),
+                        "cublas_gemms_then_unquantized_allreduce": round(ms_layer_cublas_16 * 1e3, 2)},
         "gpu_launches": args.steps, "clocks": clocks.summary()}), flush=True)
 
 
@@ -397,6 +425,7 @@ def main():
     ap.add_argument("--gemm", action="store_true",
                     help="time the tensor-core GEMM with the fused step-1 quantizer (o_proj shape)")
     ap.add_argument("--gemm-shape", type=int, nargs=3, default=[8192, 8192, 2048], metavar=("M", "N", "K"))
+    ap.add_argument("--gemm-ranks", type=int, default=4, help="ranks of the tensor-parallel layer comparison")
     ap.add_argument("--latency-sweep", action="store_true",
                     help="decode regime: per-call latency over the 16 KB .. 8 MB per rank message sweep")
     ap.add_argument("--precision-sweep", action="store_true",

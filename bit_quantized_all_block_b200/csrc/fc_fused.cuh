@@ -341,7 +341,10 @@ __global__ void __launch_bounds__(FuShape<P, SMALL>::THREADS, FuShape<P, SMALL>:
                         v = t2_bits(__hmin2(as_t2<T2>(v), as_t2<T2>(red16[r][w0 + i])));
                     u[r] = v;
                 }
-                __syncthreads();
+                // With both steps quantized, the step-2 reduction's barrier
+                // separates these reads from the next tile's writes.
+                if (B2 == 16)
+                    __syncthreads();
             }
 
             // ---- step-1 scales: one lane per rank when the group is wide enough
@@ -406,7 +409,8 @@ __global__ void __launch_bounds__(FuShape<P, SMALL>::THREADS, FuShape<P, SMALL>:
             }
             mn = fminf(mn, acc[E - 1]);
             mx = fmaxf(mx, acc[E - 1]);
-            group_minmax_f32(mn, mx, L, red32);
+            // the next tile's step-1 barrier separates these reads from the next writes
+            group_minmax_f32<B1 == 16>(mn, mx, L, red32);
             const BlockQ b2 = block_q<B2>(mn, mx);
             const bool clamp2 = __any_sync(0xffffffffu, top_code_overflows(mx, b2));
             if (valid) {
