@@ -33,6 +33,7 @@ bool valid_block(int block)
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
 
 // Byte ranges [p, p+len) for the overlap checks.
 struct Range {
@@ -96,6 +97,11 @@ const AgFnT kAg[2][2] = {
     {fc::launch_ag<__half, 8>, fc::launch_ag<__half, 4>},
     {fc::launch_ag<__nv_bfloat16, 8>, fc::launch_ag<__nv_bfloat16, 4>},
 };
+// The same with 32-byte accesses, for y and codes 32-byte aligned.
+const AgFnT kAgWide[2][2] = {
+    {fc::launch_ag<__half, 8, true>, fc::launch_ag<__half, 4, true>},
+    {fc::launch_ag<__nv_bfloat16, 8, true>, fc::launch_ag<__nv_bfloat16, 4, true>},
+};
 // [bits == 4][P - 1]
 const RsFnT kRs[2][8] = {
     {fc::launch_rs<8, 1>, fc::launch_rs<8, 2>, fc::launch_rs<8, 3>, fc::launch_rs<8, 4>,
@@ -121,6 +127,20 @@ const FusedFnT kFused[2][3][3][8] = {FC_DTYPE(__half), FC_DTYPE(__nv_bfloat16)};
 #undef FC_DTYPE
 #undef FC_P248
 #undef FC_ALLP
+// Equal quantized widths with 32-byte accesses of the inputs and the output,
+// for every x[r] and y 32-byte aligned: [dtype][bits == 4][P - 1].  Not for
+// INT8 at P = 8, where the wide form spills registers and is slower.
+#define FC_WIDE7(T, B)                                                                             \
+    fc::launch_fused<T, B, B, 1, false, true>, fc::launch_fused<T, B, B, 2, false, true>,            \
+        fc::launch_fused<T, B, B, 3, false, true>, fc::launch_fused<T, B, B, 4, false, true>,        \
+        fc::launch_fused<T, B, B, 5, false, true>, fc::launch_fused<T, B, B, 6, false, true>,        \
+        fc::launch_fused<T, B, B, 7, false, true>
+const FusedFnT kFusedWide[2][2][8] = {
+    {{FC_WIDE7(__half, 8), nullptr}, {FC_WIDE7(__half, 4), fc::launch_fused<__half, 4, 4, 8, false, true>}},
+    {{FC_WIDE7(__nv_bfloat16, 8), nullptr},
+     {FC_WIDE7(__nv_bfloat16, 4), fc::launch_fused<__nv_bfloat16, 4, 4, 8, false, true>}},
+};
+#undef FC_WIDE7
 
 int width_index(int bits) { return bits == 4 ? 0 : bits == 8 ? 1 : bits == 16 ? 2 : -1; }
 
@@ -270,7 +290,8 @@ fc_status fc_ag_dequant(const fc_qbuf* in, size_t n, int bits, int block, fc_dty
     if (any_overlap(&out, 1, ins, 3))
         return FC_ERR_INVALID_ARG;
     fc::AgArgs a{qptr(in), y, n, block};
-    cudaError_t e = kAg[out_dtype][bits == 4](a, static_cast<cudaStream_t>(stream));
+    const bool wide = aligned32(y) && aligned32(in->codes);
+    cudaError_t e = (wide ? kAgWide : kAg)[out_dtype][bits == 4](a, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? FC_OK : cuda_fail(e);
 }
 
@@ -287,7 +308,8 @@ fc_status fc_quantized_allreduce_ex(const void* const* x, int P, fc_dtype dtype,
     FusedFnT fn = kFused[dtype][w1][w2][P - 1];
     if (fn == nullptr)
         return FC_ERR_UNSUPPORTED;
-    if (FusedFnT small = small_variant(dtype, bits_rs, bits_ag, P, block, n))
+    FusedFnT small = small_variant(dtype, bits_rs, bits_ag, P, block, n);
+    if (small != nullptr)
         fn = small;
     if (n == 0)
         return FC_OK;
@@ -322,6 +344,13 @@ fc_status fc_quantized_allreduce_ex(const void* const* x, int P, fc_dtype dtype,
     }
     if (any_overlap(outs, nout, ins, P))
         return FC_ERR_INVALID_ARG;
+    if (small == nullptr && bits_rs == bits_ag && bits_rs != 16) {
+        bool wide = aligned32(y);
+        for (int r = 0; r < P; r++)
+            wide = wide && aligned32(x[r]);
+        if (wide && kFusedWide[dtype][bits_rs == 4][P - 1] != nullptr)
+            fn = kFusedWide[dtype][bits_rs == 4][P - 1];
+    }
     fc::FusedArgs a{};
     for (int r = 0; r < P; r++) {
         a.x[r] = x[r];

@@ -181,12 +181,13 @@ __device__ __forceinline__ void rank_body(const uint4* raw, const BlockQ& b, flo
 }
 
 // Step 2 on the sums, chunk by chunk: requantize, dequantize, store y (+ payload).
-template <class T, int BITS, int NC, bool CLAMP>
+template <class T, int BITS, int NC, bool CLAMP, bool WIDE>
 __device__ __forceinline__ void sum_body(const float* acc, const BlockQ& b, T* y, bool store,
                                          const QPtr& out, size_t e, bool leader, size_t k)
 {
     const float cqz = __fsub_rn(b.cq, b.zf);
     uint32_t words[NC * BITS / 4];
+    uint4 ov[NC];
 #pragma unroll
     for (int c = 0; c < NC; c++) {
         float r[8], o[8];
@@ -197,7 +198,10 @@ __device__ __forceinline__ void sum_body(const float* acc, const BlockQ& b, T* y
                 r[i] = fminf(r[i], cqz);
             o[i] = __fmul_rn(__fsub_rn(r[i], FC_MAGIC), b.s);
         }
-        st_stream(y + e + c * FC_CHUNK, narrow8<T>(o));
+        if constexpr (WIDE)
+            ov[c] = narrow8<T>(o);
+        else
+            st_stream(y + e + c * FC_CHUNK, narrow8<T>(o));
         if (store) {
             float sh[8];
 #pragma unroll
@@ -206,6 +210,8 @@ __device__ __forceinline__ void sum_body(const float* acc, const BlockQ& b, T* y
             pack_chunk<BITS>(sh, words, c);
         }
     }
+    if constexpr (WIDE)
+        store_chunks<NC, true>(y + e, ov);
     if (store) {
         store_thread_codes<BITS, NC>(out.codes, e, words);
         if (leader) {
@@ -226,12 +232,19 @@ __device__ __forceinline__ BlockQ shfl_blockq(const BlockQ& mine, int src, float
     return b;
 }
 
-template <class T, int NC>
+// Load NC chunks at p; WIDE: in pairs, one 32-byte load each (p 32-byte aligned).
+template <class T, int NC, bool WIDE = false>
 __device__ __forceinline__ void load_chunks(uint4* raw, const T* p)
 {
+    if constexpr (WIDE && NC % 2 == 0) {
 #pragma unroll
-    for (int c = 0; c < NC; c++)
-        raw[c] = ld_nc(p + c * FC_CHUNK);
+        for (int c = 0; c < NC; c += 2)
+            ld_nc_v8(p + c * FC_CHUNK, raw[c], raw[c + 1]);
+    } else {
+#pragma unroll
+        for (int c = 0; c < NC; c++)
+            raw[c] = ld_nc(p + c * FC_CHUNK);
+    }
 }
 
 // Unquantized step 1 (16-bit values sent as they are): the reduce-scatter sums
@@ -257,7 +270,9 @@ __device__ __forceinline__ void rank_body_plain(const uint4* raw, float* acc)
 // B1 / B2: bits of the reduce-scatter and of the all-gather step, each 4, 8
 // or 16 (16 = that step sends fp16/bf16 values unquantized; Fig. 5 right of
 // the page compares quantizing before RS with quantizing before AG).
-template <class T, int B1, int B2, int P, bool SMALL = false>
+// WIDE: inputs and output are moved with 32-byte accesses (every x[r] and y
+// 32-byte aligned; NC even).
+template <class T, int B1, int B2, int P, bool SMALL = false, bool WIDE = false>
 __global__ void __launch_bounds__(FuShape<P, SMALL>::THREADS, FuShape<P, SMALL>::MIN_CTAS)
     k_fused(const FusedArgs a)
 {
@@ -287,7 +302,7 @@ __global__ void __launch_bounds__(FuShape<P, SMALL>::THREADS, FuShape<P, SMALL>:
 #pragma unroll
         for (int r = 0; r < P; r++) {
             if (e0 < a.n) {
-                load_chunks<T, NC>(raw[r], static_cast<const T*>(a.x[r]) + e0);
+                load_chunks<T, NC, WIDE>(raw[r], static_cast<const T*>(a.x[r]) + e0);
             } else {
 #pragma unroll
                 for (int c = 0; c < NC; c++)
@@ -313,7 +328,7 @@ __global__ void __launch_bounds__(FuShape<P, SMALL>::THREADS, FuShape<P, SMALL>:
                 else
                     rank_body_plain<T, NC, false>(raw[r], acc);
                 if (valid_next)
-                    load_chunks<T, NC>(raw[r], static_cast<const T*>(a.x[r]) + e + stride);
+                    load_chunks<T, NC, WIDE>(raw[r], static_cast<const T*>(a.x[r]) + e + stride);
             }
         } else {
             // ---- block extremes of every rank (packed {min, -max}) ---------
@@ -387,7 +402,7 @@ __global__ void __launch_bounds__(FuShape<P, SMALL>::THREADS, FuShape<P, SMALL>:
                         rank_body<T, QB1, NC, false, false>(raw[r], b, acc, store1, a.step1[r], e, leader, k);
                 }
                 if (valid_next)   // refill rank r with the next tile while this one finishes
-                    load_chunks<T, NC>(raw[r], static_cast<const T*>(a.x[r]) + e + stride);
+                    load_chunks<T, NC, WIDE>(raw[r], static_cast<const T*>(a.x[r]) + e + stride);
             }
         }
 
@@ -395,9 +410,11 @@ __global__ void __launch_bounds__(FuShape<P, SMALL>::THREADS, FuShape<P, SMALL>:
         if constexpr (B2 == 16) {
             // ---- unquantized all-gather: the sum rounded to fp16/bf16 ----------
             if (valid) {
+                uint4 ov[NC];
 #pragma unroll
                 for (int c = 0; c < NC; c++)
-                    st_stream(y + e + c * FC_CHUNK, narrow8<T>(acc + c * FC_CHUNK));
+                    ov[c] = narrow8<T>(acc + c * FC_CHUNK);
+                store_chunks<NC, WIDE>(y + e, ov);
             }
         } else {
             // ---- step 2: requantize the sum -------------------------------------
@@ -416,9 +433,9 @@ __global__ void __launch_bounds__(FuShape<P, SMALL>::THREADS, FuShape<P, SMALL>:
             if (valid) {
                 const bool store2 = a.write_step2 != 0;
                 if (clamp2)
-                    sum_body<T, B2, NC, true>(acc, b2, y, store2, a.step2, e, leader, k);
+                    sum_body<T, B2, NC, true, WIDE>(acc, b2, y, store2, a.step2, e, leader, k);
                 else
-                    sum_body<T, B2, NC, false>(acc, b2, y, store2, a.step2, e, leader, k);
+                    sum_body<T, B2, NC, false, WIDE>(acc, b2, y, store2, a.step2, e, leader, k);
             }
         }
     }

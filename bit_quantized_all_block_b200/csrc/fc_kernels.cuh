@@ -60,8 +60,8 @@ struct FusedArgs {
 // Host-side launchers (one explicit instantiation per template in its .cu).
 template <class T, int BITS> cudaError_t launch_quantize(const QuantArgs& a, cudaStream_t st);
 template <int BITS, int P> cudaError_t launch_rs(const RsArgs& a, cudaStream_t st);
-template <class T, int BITS> cudaError_t launch_ag(const AgArgs& a, cudaStream_t st);
-template <class T, int B1, int B2, int P, bool SMALL = false>
+template <class T, int BITS, bool WIDE = false> cudaError_t launch_ag(const AgArgs& a, cudaStream_t st);
+template <class T, int B1, int B2, int P, bool SMALL = false, bool WIDE = false>
 cudaError_t launch_fused(const FusedArgs& a, cudaStream_t st);
 
 // Persistent grid: enough CTAs of `threads` threads to fill every SM at the

@@ -27,26 +27,27 @@ cudaError_t launch_rs(const RsArgs& a, cudaStream_t st)
     return cudaGetLastError();
 }
 
-template <class T, int BITS>
+template <class T, int BITS, bool WIDE>
 cudaError_t launch_ag(const AgArgs& a, cudaStream_t st)
 {
     int grid = 0;
-    cudaError_t e = persistent_grid((const void*)k_ag<T, BITS>, ST_THREADS, a.n, AgShape::TILE, &grid);
+    cudaError_t e = persistent_grid((const void*)k_ag<T, BITS, WIDE>, ST_THREADS, a.n, AgShape::TILE, &grid);
     if (e != cudaSuccess)
         return e;
-    k_ag<T, BITS><<<grid, ST_THREADS, 0, st>>>(a);
+    k_ag<T, BITS, WIDE><<<grid, ST_THREADS, 0, st>>>(a);
     return cudaGetLastError();
 }
 
-template <class T, int B1, int B2, int P, bool SMALL>
+template <class T, int B1, int B2, int P, bool SMALL, bool WIDE>
 cudaError_t launch_fused(const FusedArgs& a, cudaStream_t st)
 {
     using S = FuShape<P, SMALL>;
     int grid = 0;
-    cudaError_t e = persistent_grid((const void*)k_fused<T, B1, B2, P, SMALL>, S::THREADS, a.n, S::TILE, &grid);
+    cudaError_t e =
+        persistent_grid((const void*)k_fused<T, B1, B2, P, SMALL, WIDE>, S::THREADS, a.n, S::TILE, &grid);
     if (e != cudaSuccess)
         return e;
-    k_fused<T, B1, B2, P, SMALL><<<grid, S::THREADS, 0, st>>>(a);
+    k_fused<T, B1, B2, P, SMALL, WIDE><<<grid, S::THREADS, 0, st>>>(a);
     return cudaGetLastError();
 }
 

@@ -32,13 +32,28 @@ using QuantShape = StShape<4>;                          // 32 elements per threa
 using AgShape = StShape<4>;
 template <int P> using RsShape = StShape<(P <= 4 ? 4 : 2)>;
 
-// Load a thread's E codes (E*BITS/8 contiguous bytes) at element offset e.
-template <int BITS, int NC>
+// Load a thread's E codes (E*BITS/8 contiguous bytes) at element offset e;
+// WIDE: 32 bytes per load where there are 32 (codes 32-byte aligned).
+template <int BITS, int NC, bool WIDE = false>
 __device__ __forceinline__ void load_thread_codes(const uint8_t* codes, size_t e, uint32_t* w)
 {
     constexpr int NW = NC * BITS / 4;
     const uint8_t* p = codes + e * BITS / 8;
-    if constexpr (NW % 4 == 0) {
+    if constexpr (WIDE && NW % 8 == 0) {
+#pragma unroll
+        for (int i = 0; i < NW; i += 8) {
+            uint4 a, b;
+            ld_nc_v8(p + 4 * i, a, b);
+            w[i] = a.x;
+            w[i + 1] = a.y;
+            w[i + 2] = a.z;
+            w[i + 3] = a.w;
+            w[i + 4] = b.x;
+            w[i + 5] = b.y;
+            w[i + 6] = b.z;
+            w[i + 7] = b.w;
+        }
+    } else if constexpr (NW % 4 == 0) {
 #pragma unroll
         for (int i = 0; i < NW; i += 4) {
             const uint4 v = ld_nc(p + 4 * i);
@@ -239,8 +254,11 @@ __global__ void __launch_bounds__(ST_THREADS) k_rs(const RsArgs a)
 }
 
 // ---------------------------------------------------------------------------
-// Step 3 (all-gather): dequantize to fp16/bf16.
-template <class T, int BITS>
+// Step 3 (all-gather): dequantize to fp16/bf16.  WIDE: 32-byte stores of y
+// and (INT8) 32-byte code loads; y and the codes 32-byte aligned.  The next
+// tile's codes, scale and zero-point are loaded before the current tile is
+// dequantized and stored.
+template <class T, int BITS, bool WIDE>
 __global__ void __launch_bounds__(ST_THREADS) k_ag(const AgArgs a)
 {
     constexpr int NC = AgShape::NC, E = AgShape::E, TILE = AgShape::TILE;
@@ -249,24 +267,42 @@ __global__ void __launch_bounds__(ST_THREADS) k_ag(const AgArgs a)
     const size_t toff = (size_t)threadIdx.x * E;
     const size_t stride = (size_t)gridDim.x * TILE;
     T* y = static_cast<T*>(a.y);
-    for (size_t base = (size_t)blockIdx.x * TILE; base < a.n; base += stride) {
-        const size_t e = base + toff;
-        if (e >= a.n)
-            continue;
-        const size_t k = e >> lg_block;
-        uint32_t w[NW];
-        load_thread_codes<BITS, NC>(a.in.codes, e, w);
-        const float s = a.in.scales[k];
-        const float mz = __uint_as_float(FC_MAGIC_BITS + a.in.zps[k]);
-#pragma unroll
-        for (int c = 0; c < NC; c++) {
-            float sh[8], v[8];
-            chunk_shifted<BITS>(w, c, sh);
-#pragma unroll
-            for (int i = 0; i < 8; i++)
-                v[i] = __fmul_rn(__fsub_rn(sh[i], mz), s);
-            st_stream(y + e + c * FC_CHUNK, narrow8<T>(v));
+
+    uint32_t w[NW];
+    float s = 1.0f, mz = FC_MAGIC;
+    size_t e = (size_t)blockIdx.x * TILE + toff;
+    if (e < a.n) {
+        load_thread_codes<BITS, NC, WIDE>(a.in.codes, e, w);
+        s = a.in.scales[e >> lg_block];
+        mz = __uint_as_float(FC_MAGIC_BITS + a.in.zps[e >> lg_block]);
+    }
+    for (; e < a.n + toff; e += stride) {   // every thread of the CTA runs the same trip count
+        const size_t en = e + stride;
+        uint32_t wn[NW];
+        float sn = 1.0f, mzn = FC_MAGIC;
+        if (en < a.n) {
+            load_thread_codes<BITS, NC, WIDE>(a.in.codes, en, wn);
+            sn = a.in.scales[en >> lg_block];
+            mzn = __uint_as_float(FC_MAGIC_BITS + a.in.zps[en >> lg_block]);
         }
+        if (e < a.n) {
+            uint4 ov[NC];
+#pragma unroll
+            for (int c = 0; c < NC; c++) {
+                float sh[8], v[8];
+                chunk_shifted<BITS>(w, c, sh);
+#pragma unroll
+                for (int i = 0; i < 8; i++)
+                    v[i] = __fmul_rn(__fsub_rn(sh[i], mz), s);
+                ov[c] = narrow8<T>(v);
+            }
+            store_chunks<NC, WIDE>(y + e, ov);
+        }
+#pragma unroll
+        for (int i = 0; i < NW; i++)
+            w[i] = wn[i];
+        s = sn;
+        mz = mzn;
     }
 }
 

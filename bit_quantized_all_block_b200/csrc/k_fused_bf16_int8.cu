@@ -1,4 +1,5 @@
-// Instantiations of the fused all-reduce kernel: __nv_bfloat16, INT8 in both steps, P = 1..8.
+// Instantiations of the fused all-reduce kernel: __nv_bfloat16, INT8 in both steps, P = 1..8 with
+// 16-byte global accesses, P = 1..7 also with 32-byte ones.
 #include "fc_launch_impl.cuh"
 
 namespace fc {
@@ -10,4 +11,11 @@ template cudaError_t launch_fused<__nv_bfloat16, 8, 8, 5>(const FusedArgs&, cuda
 template cudaError_t launch_fused<__nv_bfloat16, 8, 8, 6>(const FusedArgs&, cudaStream_t);
 template cudaError_t launch_fused<__nv_bfloat16, 8, 8, 7>(const FusedArgs&, cudaStream_t);
 template cudaError_t launch_fused<__nv_bfloat16, 8, 8, 8>(const FusedArgs&, cudaStream_t);
+template cudaError_t launch_fused<__nv_bfloat16, 8, 8, 1, false, true>(const FusedArgs&, cudaStream_t);
+template cudaError_t launch_fused<__nv_bfloat16, 8, 8, 2, false, true>(const FusedArgs&, cudaStream_t);
+template cudaError_t launch_fused<__nv_bfloat16, 8, 8, 3, false, true>(const FusedArgs&, cudaStream_t);
+template cudaError_t launch_fused<__nv_bfloat16, 8, 8, 4, false, true>(const FusedArgs&, cudaStream_t);
+template cudaError_t launch_fused<__nv_bfloat16, 8, 8, 5, false, true>(const FusedArgs&, cudaStream_t);
+template cudaError_t launch_fused<__nv_bfloat16, 8, 8, 6, false, true>(const FusedArgs&, cudaStream_t);
+template cudaError_t launch_fused<__nv_bfloat16, 8, 8, 7, false, true>(const FusedArgs&, cudaStream_t);
 }  // namespace fc

@@ -1,4 +1,5 @@
-// Instantiations of the fused all-reduce kernel: __half, INT4 in both steps, P = 1..8.
+// Instantiations of the fused all-reduce kernel: __half, INT4 in both steps, P = 1..8, with
+// 16-byte and with 32-byte global accesses.
 #include "fc_launch_impl.cuh"
 
 namespace fc {
@@ -10,4 +11,12 @@ template cudaError_t launch_fused<__half, 4, 4, 5>(const FusedArgs&, cudaStream_
 template cudaError_t launch_fused<__half, 4, 4, 6>(const FusedArgs&, cudaStream_t);
 template cudaError_t launch_fused<__half, 4, 4, 7>(const FusedArgs&, cudaStream_t);
 template cudaError_t launch_fused<__half, 4, 4, 8>(const FusedArgs&, cudaStream_t);
+template cudaError_t launch_fused<__half, 4, 4, 1, false, true>(const FusedArgs&, cudaStream_t);
+template cudaError_t launch_fused<__half, 4, 4, 2, false, true>(const FusedArgs&, cudaStream_t);
+template cudaError_t launch_fused<__half, 4, 4, 3, false, true>(const FusedArgs&, cudaStream_t);
+template cudaError_t launch_fused<__half, 4, 4, 4, false, true>(const FusedArgs&, cudaStream_t);
+template cudaError_t launch_fused<__half, 4, 4, 5, false, true>(const FusedArgs&, cudaStream_t);
+template cudaError_t launch_fused<__half, 4, 4, 6, false, true>(const FusedArgs&, cudaStream_t);
+template cudaError_t launch_fused<__half, 4, 4, 7, false, true>(const FusedArgs&, cudaStream_t);
+template cudaError_t launch_fused<__half, 4, 4, 8, false, true>(const FusedArgs&, cudaStream_t);
 }  // namespace fc

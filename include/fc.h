@@ -47,7 +47,10 @@
  *     bits must be 4 or 8; block a power of two in [32, 4096]; P in [1, 8];
  *     n a multiple of block (and of P*block where chunks are involved).
  *     n == 0 is a no-op returning FC_OK (pointers are then not inspected).
- *     Every device pointer must be non-NULL and 16-byte aligned.
+ *     Every device pointer must be non-NULL and 16-byte aligned.  When the
+ *     inputs and the output are also 32-byte aligned, the fused all-reduce
+ *     (equal widths) and the all-gather step move them with 32-byte accesses,
+ *     which is faster; the results are the same bits either way.
  *     Output buffers must not overlap input buffers (checked).
  *   - Inputs must be finite.  For bf16, every block whose range is nonzero
  *     must have a range in [2^-100, 2^100]; outside that the scale or its

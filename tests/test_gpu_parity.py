@@ -111,3 +111,57 @@ def test_staged_and_fused_calls_on_a_side_stream():
         y = fc.fc_quantized_allreduce(xd, 8, 128)
     s.synchronize()
     assert_y_equal(y, y_ref, "side stream")
+
+
+def _at_16_mod_32(t):
+    """A copy of t whose data pointer is 16-byte but not 32-byte aligned."""
+    pad = 32 // t.element_size()
+    buf = torch.empty(t.numel() + pad, dtype=t.dtype, device=t.device)
+    v = buf[pad // 2: pad // 2 + t.numel()]
+    assert v.data_ptr() % 32 == 16
+    v.copy_(t)
+    return v
+
+
+def _qbuf_at_16_mod_32(n, bits, block):
+    q = fc.QBuf.empty(n, bits, block)
+    return fc.QBuf(_at_16_mod_32(q.codes), _at_16_mod_32(q.scales), _at_16_mod_32(q.zps), n, bits, block)
+
+
+@pytest.mark.parametrize("dtype", [oracle.FP16, oracle.BF16], ids=["fp16", "bf16"])
+@pytest.mark.parametrize("bits", [8, 4])
+@pytest.mark.parametrize("block", [32, 128, 1024])
+@pytest.mark.parametrize("P", [1, 2, 3, 4, 8])
+@pytest.mark.parametrize("which", ["all", "y", "x_last"])
+def test_buffers_aligned_to_16_but_not_32(dtype, bits, block, P, which):
+    """The kernels move 32 bytes per access when every pointer allows it and
+    16 bytes otherwise; both forms give the oracle's bits.  `which` names the
+    buffers placed at an address that is 16 mod 32."""
+    m = (2 * 4096) // (P * block) + 3
+    n = P * block * m
+    xs = synth.partials(P, n // block, block, dtype, 0.05, 20.0, seed=900 + block + P + bits)
+    y_ref, p1_ref, p2_ref = oracle.allreduce(list(xs), dtype, bits, block)
+    xd = to_dev(xs, dtype)
+    if which in ("all", "x_last"):
+        xd[-1] = _at_16_mod_32(xd[-1])
+    if which == "all":
+        xd = [_at_16_mod_32(x) for x in xd]
+    y = torch.empty(n, dtype=tdtype(dtype), device="cuda")
+    if which in ("all", "y"):
+        y = _at_16_mod_32(y)
+    mk = _qbuf_at_16_mod_32 if which == "all" else fc.QBuf.empty
+    s1 = [mk(n, bits, block) for _ in range(P)]
+    s2 = mk(n, bits, block)
+    fc.fc_quantized_allreduce(xd, bits, block, y=y, step1=s1, step2=s2)
+    torch.cuda.synchronize()
+    assert_y_equal(y, y_ref, f"fused y ({which})")
+    for r in range(P):
+        assert_payload_equal(s1[r], p1_ref[r], f"fused step1[{r}] ({which})")
+    assert_payload_equal(s2, p2_ref, f"fused step2 ({which})")
+    # the all-gather step alone, reading the payload just written
+    y2 = torch.empty(n, dtype=tdtype(dtype), device="cuda")
+    if which in ("all", "y"):
+        y2 = _at_16_mod_32(y2)
+    fc.fc_ag_dequant(s2, tdtype(dtype), y=y2)
+    torch.cuda.synchronize()
+    assert_y_equal(y2, y_ref, f"staged y ({which})")
