@@ -71,6 +71,11 @@ def _lib():
         for f in ("fc_payload_sizes", "fc_quantize", "fc_rs_dequant_sum_requant", "fc_ag_dequant",
                   "fc_quantized_allreduce", "fc_quantized_allreduce_ex", "fc_gemm_quantize"):
             getattr(L, f).restype = I
+        L.fc_ipc_export.argtypes = [P, ctypes.c_char_p, ctypes.POINTER(S)]
+        L.fc_ipc_open.argtypes = [ctypes.c_char_p, ctypes.POINTER(P)]
+        L.fc_ipc_close.argtypes = [P]
+        for f in ("fc_ipc_export", "fc_ipc_open", "fc_ipc_close"):
+            getattr(L, f).restype = I
         L.fc_status_string.argtypes = [I]
         L.fc_status_string.restype = ctypes.c_char_p
         L.fc_last_cuda_error.argtypes = []
@@ -152,6 +157,42 @@ class QBuf:
 
     def bytes(self) -> int:
         return self.codes.numel() + 4 * self.scales.numel() + self.zps.numel()
+
+
+class PeerQBuf(QBuf):
+    """A payload held by another process's GPU, seen through fc_ipc_open
+    mappings: raw device addresses instead of tensors."""
+
+    def __init__(self, codes: int, scales: int, zps: int, n: int, bits: int, block: int):
+        self.codes, self.scales, self.zps = codes, scales, zps
+        self.n, self.bits, self.block = n, bits, block
+
+    def struct(self):
+        return fc_qbuf(self.codes, self.scales, self.zps)
+
+
+FC_IPC_HANDLE_BYTES = 64
+
+
+def fc_ipc_export(ptr: int) -> tuple[bytes, int]:
+    """(IPC handle of the allocation holding device address ``ptr``, ptr's offset in it)."""
+    h = ctypes.create_string_buffer(FC_IPC_HANDLE_BYTES)
+    off = ctypes.c_size_t()
+    _check(_lib().fc_ipc_export(ctypes.c_void_p(ptr), h, ctypes.byref(off)), "fc_ipc_export")
+    return h.raw, off.value
+
+
+def fc_ipc_open(handle: bytes) -> int:
+    """Map another process's exported allocation; returns the base address."""
+    if len(handle) != FC_IPC_HANDLE_BYTES:
+        raise ValueError("an IPC handle is 64 bytes")
+    base = ctypes.c_void_p()
+    _check(_lib().fc_ipc_open(handle, ctypes.byref(base)), "fc_ipc_open")
+    return base.value
+
+
+def fc_ipc_close(base: int) -> None:
+    _check(_lib().fc_ipc_close(ctypes.c_void_p(base)), "fc_ipc_close")
 
 
 def fc_quantize(x, bits: int, block: int, out: QBuf | None = None, stream=None) -> QBuf:

@@ -7,6 +7,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <cstring>
 #include <map>
 #include <mutex>
 #include <utility>
@@ -242,8 +243,9 @@ fc_status fc_quantize(const void* x, fc_dtype dtype, size_t n, int bits, int blo
 fc_status fc_rs_dequant_sum_requant(const fc_qbuf* in, int P, size_t n, int bits, int block,
                                     const fc_qbuf* out, void* stream)
 {
-    if (!valid_bits(bits) || !valid_block(block) || P < 1 || P > fc::FC_MAX_P ||
-        n % ((size_t)P * (size_t)block) != 0)
+    // Each block of the sum depends only on the same block of every rank, so
+    // any whole number of blocks is a valid range (one owner's chunk included).
+    if (!valid_bits(bits) || !valid_block(block) || P < 1 || P > fc::FC_MAX_P || n % (size_t)block != 0)
         return FC_ERR_INVALID_ARG;
     if (n == 0)
         return FC_OK;
@@ -490,6 +492,55 @@ fc_status fc_gemm_quantize(const void* a, const void* w, fc_dtype dtype, int M, 
         return cuda_fail(e);
     const int bi = block == 32 ? 0 : block == 64 ? 1 : 2;
     e = (pair ? kGemmPair : kGemm)[dtype][qbits == 4][bi](ta, tb, g, st);
+    return e == cudaSuccess ? FC_OK : cuda_fail(e);
+}
+
+// ---- peer memory (CUDA IPC) for the P-GPU deployment -------------------------
+static_assert(sizeof(cudaIpcMemHandle_t) == FC_IPC_HANDLE_BYTES, "IPC handle size");
+
+fc_status fc_ipc_export(const void* ptr, void* handle, size_t* offset)
+{
+    if (ptr == nullptr || handle == nullptr || offset == nullptr)
+        return FC_ERR_INVALID_ARG;
+    static PFN_cuMemGetAddressRange range = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuMemGetAddressRange", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            range = reinterpret_cast<PFN_cuMemGetAddressRange>(p);
+    });
+    if (range == nullptr)
+        return cuda_fail(cudaErrorNotSupported);
+    CUdeviceptr base = 0;
+    size_t size = 0;
+    if (range(&base, &size, reinterpret_cast<CUdeviceptr>(ptr)) != CUDA_SUCCESS)
+        return FC_ERR_INVALID_ARG;   // not device memory of the current context
+    cudaIpcMemHandle_t h;
+    cudaError_t e = cudaIpcGetMemHandle(&h, reinterpret_cast<void*>(base));
+    if (e != cudaSuccess)
+        return cuda_fail(e);
+    memcpy(handle, &h, sizeof(h));
+    *offset = reinterpret_cast<uintptr_t>(ptr) - static_cast<uintptr_t>(base);
+    return FC_OK;
+}
+
+fc_status fc_ipc_open(const void* handle, void** base)
+{
+    if (handle == nullptr || base == nullptr)
+        return FC_ERR_INVALID_ARG;
+    cudaIpcMemHandle_t h;
+    memcpy(&h, handle, sizeof(h));
+    cudaError_t e = cudaIpcOpenMemHandle(base, h, cudaIpcMemLazyEnablePeerAccess);
+    return e == cudaSuccess ? FC_OK : cuda_fail(e);
+}
+
+fc_status fc_ipc_close(void* base)
+{
+    if (base == nullptr)
+        return FC_ERR_INVALID_ARG;
+    cudaError_t e = cudaIpcCloseMemHandle(base);
     return e == cudaSuccess ? FC_OK : cuda_fail(e);
 }
 

@@ -104,7 +104,11 @@ fc_status fc_quantize(const void* x, fc_dtype dtype, size_t n, int bits, int blo
  * owner's work is done: dequantize chunk c from all P payloads, sum in fp32 in
  * rank order 0..P-1, requantize.  *out receives the step-2 payload of all n
  * elements (chunk c at its natural offset, so the P owners' outputs form one
- * payload).  Requires n % (P*block) == 0. */
+ * payload).  Every block of the result depends only on the same block of the
+ * P inputs, so any block-aligned range is valid: one owner of a P-GPU
+ * all-reduce passes, for its chunk only, the P ranks' step-1 payload pointers
+ * offset to that chunk (peer pointers from fc_ipc_open), n = the chunk length.
+ * Requires n % block == 0 (n % (P*block) == 0 for P equal chunks). */
 fc_status fc_rs_dequant_sum_requant(const fc_qbuf* in, int P, size_t n, int bits, int block,
                                     const fc_qbuf* out, void* stream);
 
@@ -169,6 +173,33 @@ fc_status fc_quantized_allreduce_ex(const void* const* x, int P, fc_dtype dtype,
  * persistent kernel (one CTA per SM, 197 KB shared memory, 512 TMEM columns). */
 fc_status fc_gemm_quantize(const void* a, const void* w, fc_dtype dtype, int M, int N, int K, int bits, int block,
                            const fc_qbuf* out, void* partial, int* status, void* stream);
+
+/* Peer memory for the P-GPU deployment (one process per GPU; the page's
+ * setting, Fig. 1 and Fig. 3: each rank's payloads live in its own GPU and
+ * the other ranks read them over NVLink).  A rank exports the device buffers
+ * that hold its payloads; every other rank maps them and passes the mapped
+ * pointers to fc_rs_dequant_sum_requant / fc_ag_dequant, whose loads then
+ * read the peer's memory directly.  These calls map memory and create no
+ * buffers; they synchronize nothing.  Memory from the stream-ordered
+ * allocator or from virtual-memory-management reservations cannot be
+ * exported (FC_ERR_CUDA). */
+#define FC_IPC_HANDLE_BYTES 64
+
+/* Export the device allocation that contains ptr: writes its 64-byte CUDA
+ * IPC handle to handle (host memory) and ptr's byte offset inside it to
+ * *offset.  Errors: FC_ERR_INVALID_ARG for NULL arguments or a pointer that
+ * is not device memory of the current context; FC_ERR_CUDA. */
+fc_status fc_ipc_export(const void* ptr, void* handle, size_t* offset);
+
+/* Map an allocation exported by another process (not this one) into this
+ * process on the current device, enabling peer access if it lives on another
+ * GPU; *base receives the mapping (the exporter's ptr is *base + offset).
+ * Errors: FC_ERR_INVALID_ARG for NULL arguments; FC_ERR_CUDA. */
+fc_status fc_ipc_open(const void* handle, void** base);
+
+/* Unmap a base returned by fc_ipc_open (after all work that reads it has
+ * completed).  Errors: FC_ERR_INVALID_ARG for NULL; FC_ERR_CUDA. */
+fc_status fc_ipc_close(void* base);
 
 /* Static description of a status code. */
 const char* fc_status_string(fc_status status);

@@ -98,8 +98,24 @@ def test_staged_validation():
     assert lib.fc_quantize(ctypes.c_void_p(A), 0, 4096, 8, 128, ctypes.byref(qo), None) == fc.FC_ERR_INVALID_ARG
     ins = (fc.fc_qbuf * 2)(qb(A), qb(A + 0x4000000))
     assert lib.fc_rs_dequant_sum_requant(ins, 2, 4096, 8, 128, ctypes.byref(ins[0]), None) == fc.FC_ERR_INVALID_ARG
-    assert lib.fc_rs_dequant_sum_requant(ins, 2, 4096 + 128, 8, 128, ctypes.byref(q), None) == fc.FC_ERR_INVALID_ARG
+    # any whole number of blocks is a valid range; a partial block is not
+    assert lib.fc_rs_dequant_sum_requant(ins, 2, 4096 + 64, 8, 128, ctypes.byref(q), None) == fc.FC_ERR_INVALID_ARG
     assert lib.fc_rs_dequant_sum_requant(ins, 2, 0, 8, 128, None, None) == fc.FC_OK
     assert lib.fc_ag_dequant(ctypes.byref(q), 4096, 8, 128, 0, ctypes.c_void_p(A + 0x50000000), None) == fc.FC_ERR_INVALID_ARG
     assert lib.fc_ag_dequant(ctypes.byref(q), 4096, 8, 128, 0, ctypes.c_void_p(A + 0x7000000a), None) == fc.FC_ERR_MISALIGNED
     assert lib.fc_ag_dequant(ctypes.byref(q), 4096, 8, 128, 3, ctypes.c_void_p(A), None) == fc.FC_ERR_INVALID_ARG
+
+
+def test_ipc_validation():
+    lib = fc.library()
+    h = ctypes.create_string_buffer(fc.FC_IPC_HANDLE_BYTES)
+    off = ctypes.c_size_t()
+    base = ctypes.c_void_p()
+    assert lib.fc_ipc_export(None, h, ctypes.byref(off)) == fc.FC_ERR_INVALID_ARG
+    assert lib.fc_ipc_export(ctypes.c_void_p(A), None, ctypes.byref(off)) == fc.FC_ERR_INVALID_ARG
+    assert lib.fc_ipc_export(ctypes.c_void_p(A), h, None) == fc.FC_ERR_INVALID_ARG
+    assert lib.fc_ipc_open(None, ctypes.byref(base)) == fc.FC_ERR_INVALID_ARG
+    assert lib.fc_ipc_open(h, None) == fc.FC_ERR_INVALID_ARG
+    assert lib.fc_ipc_close(None) == fc.FC_ERR_INVALID_ARG
+    with pytest.raises(ValueError):
+        fc.fc_ipc_open(b"short")

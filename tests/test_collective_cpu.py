@@ -1,0 +1,86 @@
+"""The P-rank quantized all-reduce's host logic on CPU (no GPU): arena layout,
+the per-rank schedule, and the whole three-step exchange run by 2 and 4 gloo
+ranks (one process each) whose arenas are shared memory and whose steps are
+the oracle's -- the result must be the oracle's one-process all-reduce, bit
+for bit, on every rank, over two consecutive calls on the same arenas."""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import oracle
+from bit_quantized_all_block_b200 import synth
+from bit_quantized_all_block_b200.collective import ALIGN, Layout, QuantizedAllReduce, schedule
+
+
+@pytest.mark.parametrize("n,P,bits,block", [(4096, 2, 8, 128), (4096, 4, 4, 32), (65536, 8, 4, 4096),
+                                            (3 * 8 * 512, 8, 8, 512)])
+def test_layout_parts_are_aligned_sized_and_disjoint(n, P, bits, block):
+    L = Layout(n, P, bits, block)
+    m = n // P
+    parts = []
+    for ref in [L.step1(0, c) for c in range(P)] + [L.step2(0)]:
+        assert ref.n == m
+        parts += [(ref.codes, m * bits // 8), (ref.scales, 4 * (m // block)), (ref.zps, m // block)]
+    for off, size in parts:
+        assert off % ALIGN == 0 and off + size <= L.nbytes
+    parts.sort()
+    for (o1, s1), (o2, _) in zip(parts, parts[1:]):
+        assert o1 + s1 <= o2
+
+
+def test_layout_rejects_chunks_that_are_not_whole_blocks():
+    with pytest.raises(ValueError):
+        Layout(4096 + 128, 2, 8, 128)
+
+
+def test_schedule_reads_the_owned_chunk_from_every_rank():
+    L = Layout(8192, 4, 8, 128)
+    for rank in range(4):
+        quantize, (ins, out), ag = schedule(rank, L)
+        assert [q.holder for q in quantize] == [rank] * 4
+        assert quantize == [L.step1(rank, c) for c in range(4)]
+        assert ins == [L.step1(r, rank) for r in range(4)]       # chunk `rank` of every holder
+        assert out == L.step2(rank)
+        assert [a.holder for a in ag] == [0, 1, 2, 3]
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, case, out):
+    from tests.collective_cpu_ops import OracleOps
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        n, dtype, bits, block, seeds = case
+        ar = QuantizedAllReduce(n, bits, block, ops=OracleOps(dtype))
+        ys = []
+        for seed in seeds:
+            xs = synth.partials(world, n // block, block, dtype, 0.05, 20.0, seed=seed)
+            ys.append(ar(xs[rank]).copy())
+        ar.close()
+        out[rank] = ys
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,bits,block,dtype", [(2, 8, 128, oracle.FP16), (4, 4, 64, oracle.BF16)])
+def test_ranks_reproduce_the_one_process_allreduce(world, bits, block, dtype):
+    n = world * world * block * 3     # the oracle's RS step wants whole P-block groups per chunk
+    seeds = (11, 12)
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    mp.start_processes(_rank_main, args=(world, _free_port(), (n, dtype, bits, block, seeds), out),
+                       nprocs=world, join=True, start_method="spawn")
+    for k, seed in enumerate(seeds):
+        xs = synth.partials(world, n // block, block, dtype, 0.05, 20.0, seed=seed)
+        y_ref, _, _ = oracle.allreduce(list(xs), dtype, bits, block)
+        for r in range(world):
+            assert np.array_equal(out[r][k], y_ref), f"rank {r}, call {k}"

@@ -165,3 +165,30 @@ def test_buffers_aligned_to_16_but_not_32(dtype, bits, block, P, which):
     fc.fc_ag_dequant(s2, tdtype(dtype), y=y2)
     torch.cuda.synchronize()
     assert_y_equal(y2, y_ref, f"staged y ({which})")
+
+
+@pytest.mark.parametrize("bits", [8, 4])
+@pytest.mark.parametrize("P", [2, 3, 8])
+def test_reduce_scatter_on_a_block_range(bits, P):
+    """Every block of the reduce-scatter depends only on the same block of the
+    P inputs, so the call on any block-aligned range (pointers offset into the
+    payloads, a length that need not be a multiple of P blocks -- one owner's
+    chunk in a P-GPU run) gives those blocks of the whole call."""
+    block, nblk, k0, k = 64, 48, 16, 5
+    n = nblk * block
+    xs = synth.partials(P, nblk, block, oracle.FP16, 0.05, 20.0, seed=40 + P + bits)
+    p1 = [oracle.quantize(x, oracle.FP16, bits, block) for x in xs]
+    p2 = oracle.rs_dequant_sum_requant(p1)
+    dev = [fc.QBuf(torch.from_numpy(p.codes).cuda(), torch.from_numpy(p.scales).cuda(),
+                   torch.from_numpy(p.zps).cuda(), n, bits, block) for p in p1]
+    cb = block * bits // 8
+
+    def sub(q):
+        return fc.PeerQBuf(q.codes.data_ptr() + k0 * cb, q.scales.data_ptr() + 4 * k0, q.zps.data_ptr() + k0,
+                           k * block, bits, block)
+    out = fc.QBuf.empty(k * block, bits, block)
+    fc.fc_rs_dequant_sum_requant([sub(q) for q in dev], bits, block, out=out)
+    torch.cuda.synchronize()
+    assert np.array_equal(out.codes.cpu().numpy(), p2.codes[k0 * cb:(k0 + k) * cb])
+    assert np.array_equal(out.scales.cpu().numpy().view(np.uint32), p2.scales[k0:k0 + k].view(np.uint32))
+    assert np.array_equal(out.zps.cpu().numpy(), p2.zps[k0:k0 + k])
