@@ -538,16 +538,16 @@ def main():
 
     variants = args.variant.split(",")
     for vi, variant in enumerate(variants):
-        def step():
+        def step(xs_=xs, y_=y):
             if variant == "fused":
-                fc.fc_quantized_allreduce(xs, w.bits, w.block, y=y, step1=s1, step2=s2)
+                fc.fc_quantized_allreduce(xs_, w.bits, w.block, y=y_, step1=s1, step2=s2)
             elif variant == "fused_nopayload":
-                fc.fc_quantized_allreduce(xs, w.bits, w.block, y=y)
+                fc.fc_quantized_allreduce(xs_, w.bits, w.block, y=y_)
             else:
                 for r in range(w.P):
-                    fc.fc_quantize(xs[r], w.bits, w.block, out=s1[r])
+                    fc.fc_quantize(xs_[r], w.bits, w.block, out=s1[r])
                 fc.fc_rs_dequant_sum_requant(s1, w.bits, w.block, out=s2)
-                fc.fc_ag_dequant(s2, tdt, y=y)
+                fc.fc_ag_dequant(s2, tdt, y=y_)
 
         launches_per_step = 1 if variant.startswith("fused") else w.P + 2
 
@@ -622,24 +622,42 @@ def main():
         ms = max_over_ranks(ms, world)
 
         # ---- end to end through the public API with host buffers -----------------
+        # The same calls on the page-locked host inputs and a page-locked host
+        # output: the kernels read the inputs from host memory and write the
+        # result there themselves (zero-copy through the bus), so every step's
+        # host->device and device->host traffic is inside the timed region.
+        # The explicit-copy form (asynchronous copies of the inputs, the call on
+        # device buffers, a copy of the result back) is timed beside it.
         y_host = torch.empty(w.n, dtype=tdt).pin_memory()
-        for _ in range(2):
+
+        def e2e_copies():
             for r in range(w.P):
                 xs[r].copy_(xs_pinned[r], non_blocking=True)
             step()
             y_host.copy_(y, non_blocking=True)
-        torch.cuda.synchronize()
-        barrier()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(args.e2e_steps):
-            for r in range(w.P):
-                xs[r].copy_(xs_pinned[r], non_blocking=True)
-            step()
-            y_host.copy_(y, non_blocking=True)
-        e1.record(stream)
-        torch.cuda.synchronize()
-        ms_e2e = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, world)
+
+        def e2e_zero_copy():
+            step(xs_pinned, y_host)
+
+        def time_e2e(fn):
+            for _ in range(2):
+                fn()
+            torch.cuda.synchronize()
+            barrier()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(args.e2e_steps):
+                fn()
+            b.record(stream)
+            torch.cuda.synchronize()
+            return max_over_ranks(a.elapsed_time(b) / args.e2e_steps, world)
+
+        ms_copies = time_e2e(e2e_copies)
+        ms_zero = time_e2e(e2e_zero_copy)
+        e2e_exact = bool(torch.equal(y_host.view(torch.int16), y.view(torch.int16).cpu()))
+        # the headline e2e figure is the faster of the two ways a user can call the library
+        zero_wins = ms_zero <= ms_copies
+        ms_e2e = ms_zero if zero_wins else ms_copies
 
         in_bytes = w.P * w.n * 2
         value = job_throughput(in_bytes, world, ms)
@@ -667,6 +685,11 @@ def main():
                          "algorithmic_bytes_per_launch": alg if variant.startswith("fused") else None,
                          "algorithmic_bytes_per_step": alg},
             "e2e": {"value": round(value_e2e, 3), "unit": "GB/s", "h2d_bytes_per_step": in_bytes,
+                    "mode": ("zero-copy: the call on page-locked host buffers" if zero_wins else
+                             "explicit copies: H2D of the inputs, the call on device buffers, D2H of the result"),
+                    "zero_copy_value": round(job_throughput(in_bytes, world, ms_zero), 3),
+                    "explicit_copies_value": round(job_throughput(in_bytes, world, ms_copies), 3),
+                    "zero_copy_output_equals_device_path": e2e_exact,
                     "d2h_bytes_per_step": w.n * 2},
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clocks.summary(),

@@ -71,6 +71,8 @@ def _lib():
         for f in ("fc_payload_sizes", "fc_quantize", "fc_rs_dequant_sum_requant", "fc_ag_dequant",
                   "fc_quantized_allreduce", "fc_quantized_allreduce_ex", "fc_gemm_quantize"):
             getattr(L, f).restype = I
+        L.fc_host_device_pointer.argtypes = [P, ctypes.POINTER(P)]
+        L.fc_host_device_pointer.restype = I
         L.fc_ipc_export.argtypes = [P, ctypes.c_char_p, ctypes.POINTER(S)]
         L.fc_ipc_open.argtypes = [ctypes.c_char_p, ctypes.POINTER(P)]
         L.fc_ipc_close.argtypes = [P]
@@ -125,9 +127,30 @@ def _stream(stream):
 
 
 def _dev_ptr(t, name: str) -> int:
-    if not t.is_cuda or not t.is_contiguous():
-        raise ValueError(f"{name} must be a contiguous CUDA tensor")
-    return t.data_ptr()
+    """Device address of a contiguous CUDA tensor, or of a contiguous page-locked
+    CPU tensor (the kernels then access host memory directly)."""
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.is_cuda:
+        return t.data_ptr()
+    if t.device.type == "cpu" and t.is_pinned():
+        return fc_host_device_pointer(t.data_ptr())
+    raise ValueError(f"{name} must be a CUDA tensor or a page-locked (pinned) CPU tensor")
+
+
+def fc_host_device_pointer(host_ptr: int) -> int:
+    """Device address of mapped page-locked host memory at ``host_ptr``."""
+    d = ctypes.c_void_p()
+    _check(_lib().fc_host_device_pointer(ctypes.c_void_p(host_ptr), ctypes.byref(d)), "fc_host_device_pointer")
+    return d.value
+
+
+def _new_like(t, n: int):
+    """An output of n elements next to t: on its GPU, or page-locked if t is a pinned CPU tensor."""
+    import torch
+    if t.is_cuda:
+        return torch.empty(n, dtype=t.dtype, device=t.device)
+    return torch.empty(n, dtype=t.dtype).pin_memory()
 
 
 def fc_payload_sizes(n: int, bits: int, block: int) -> tuple[int, int]:
@@ -198,7 +221,7 @@ def fc_ipc_close(base: int) -> None:
 def fc_quantize(x, bits: int, block: int, out: QBuf | None = None, stream=None) -> QBuf:
     """Step 1 on one rank: quantize the fp16/bf16 tensor x (flattened)."""
     n = x.numel()
-    out = out or QBuf.empty(n, bits, block, x.device)
+    out = out or QBuf.empty(n, bits, block, x.device if x.is_cuda else "cuda")
     q = out.struct()
     _check(_lib().fc_quantize(ctypes.c_void_p(_dev_ptr(x, "x")), _dtype_code(x), n, bits, block,
                               ctypes.byref(q), _stream(stream)), "fc_quantize")
@@ -209,7 +232,7 @@ def fc_rs_dequant_sum_requant(ins, bits: int, block: int, out: QBuf | None = Non
     """Reduce-scatter step over the P step-1 payloads ``ins``; returns the step-2 payload."""
     P = len(ins)
     n = ins[0].n
-    out = out or QBuf.empty(n, bits, block, ins[0].codes.device)
+    out = out or QBuf.empty(n, bits, block, ins[0].codes.device if hasattr(ins[0].codes, "device") else "cuda")
     arr = (fc_qbuf * P)(*[q.struct() for q in ins])
     q2 = out.struct()
     _check(_lib().fc_rs_dequant_sum_requant(arr, P, n, bits, block, ctypes.byref(q2), _stream(stream)),
@@ -223,7 +246,9 @@ def fc_ag_dequant(q: QBuf, out_dtype, y=None, stream=None):
     code = FC_FP16 if out_dtype == torch.float16 else FC_BF16 if out_dtype == torch.bfloat16 else None
     if code is None:
         raise TypeError(f"out_dtype must be float16 or bfloat16, got {out_dtype}")
-    y = torch.empty(q.n, dtype=out_dtype, device=q.codes.device) if y is None else y
+    if y is None:
+        dev = q.codes.device if hasattr(q.codes, "device") else "cuda"
+        y = torch.empty(q.n, dtype=out_dtype, device=dev)
     qs = q.struct()
     _check(_lib().fc_ag_dequant(ctypes.byref(qs), q.n, q.bits, q.block, code,
                                 ctypes.c_void_p(_dev_ptr(y, "y")), _stream(stream)), "fc_ag_dequant")
@@ -242,7 +267,7 @@ def fc_quantized_allreduce(xs, bits: int, block: int, y=None, step1=None, step2:
     for x in xs:
         if x.numel() != n or _dtype_code(x) != dt:
             raise ValueError("all partials must have the same size and dtype")
-    y = torch.empty(n, dtype=xs[0].dtype, device=xs[0].device) if y is None else y
+    y = _new_like(xs[0], n) if y is None else y
     xp = (ctypes.c_void_p * P)(*[_dev_ptr(x, "x") for x in xs])
     s1 = (fc_qbuf * P)(*[q.struct() for q in step1]) if step1 is not None else None
     s2 = step2.struct() if step2 is not None else None
@@ -262,7 +287,7 @@ def fc_quantized_allreduce_ex(xs, bits_rs: int, bits_ag: int, block: int, y=None
     for x in xs:
         if x.numel() != n or _dtype_code(x) != dt:
             raise ValueError("all partials must have the same size and dtype")
-    y = torch.empty(n, dtype=xs[0].dtype, device=xs[0].device) if y is None else y
+    y = _new_like(xs[0], n) if y is None else y
     xp = (ctypes.c_void_p * P)(*[_dev_ptr(x, "x") for x in xs])
     s1 = (fc_qbuf * P)(*[q.struct() for q in step1]) if step1 is not None else None
     s2 = step2.struct() if step2 is not None else None

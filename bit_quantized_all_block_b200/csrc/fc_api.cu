@@ -495,6 +495,20 @@ fc_status fc_gemm_quantize(const void* a, const void* w, fc_dtype dtype, int M, 
     return e == cudaSuccess ? FC_OK : cuda_fail(e);
 }
 
+fc_status fc_host_device_pointer(const void* host, void** device)
+{
+    if (host == nullptr || device == nullptr)
+        return FC_ERR_INVALID_ARG;
+    void* d = nullptr;
+    cudaError_t e = cudaHostGetDevicePointer(&d, const_cast<void*>(host), 0);
+    if (e != cudaSuccess || d == nullptr) {
+        cudaGetLastError();   // not mapped page-locked memory; keep the error out of later launch checks
+        return FC_ERR_INVALID_ARG;
+    }
+    *device = d;
+    return FC_OK;
+}
+
 // ---- peer memory (CUDA IPC) for the P-GPU deployment -------------------------
 static_assert(sizeof(cudaIpcMemHandle_t) == FC_IPC_HANDLE_BYTES, "IPC handle size");
 

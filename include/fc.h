@@ -37,7 +37,10 @@
  *
  * Conventions for every entry point:
  *   - Pointers named as device pointers must be CUDA device memory (or
- *     managed memory) of the current device; arrays of pointers and the
+ *     managed memory) of the current device, or page-locked host memory
+ *     mapped into the device's address space, given by its device address
+ *     (fc_host_device_pointer); the kernels then read and write that host
+ *     memory over the bus themselves (zero-copy).  Arrays of pointers and the
  *     fc_qbuf structs themselves live in host memory and are read before the
  *     call returns.  The caller owns every buffer; the library allocates
  *     nothing and keeps no reference after the call.
@@ -173,6 +176,15 @@ fc_status fc_quantized_allreduce_ex(const void* const* x, int P, fc_dtype dtype,
  * persistent kernel (one CTA per SM, 197 KB shared memory, 512 TMEM columns). */
 fc_status fc_gemm_quantize(const void* a, const void* w, fc_dtype dtype, int M, int N, int K, int bits, int block,
                            const fc_qbuf* out, void* partial, int* status, void* stream);
+
+/* The device address of page-locked host memory that is mapped into the
+ * device's address space (memory from cudaHostAlloc -- every such allocation
+ * is mapped under unified addressing -- or registered with the mapped flag).
+ * Passing that address to the entry points above lets a kernel stream its
+ * inputs from, or its outputs to, host memory directly.  Host only.
+ * Errors: FC_ERR_INVALID_ARG for NULL arguments or memory that is not mapped
+ * page-locked host memory. */
+fc_status fc_host_device_pointer(const void* host, void** device);
 
 /* Peer memory for the P-GPU deployment (one process per GPU; the page's
  * setting, Fig. 1 and Fig. 3: each rank's payloads live in its own GPU and

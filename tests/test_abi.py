@@ -117,5 +117,8 @@ def test_ipc_validation():
     assert lib.fc_ipc_open(None, ctypes.byref(base)) == fc.FC_ERR_INVALID_ARG
     assert lib.fc_ipc_open(h, None) == fc.FC_ERR_INVALID_ARG
     assert lib.fc_ipc_close(None) == fc.FC_ERR_INVALID_ARG
+    dev = ctypes.c_void_p()
+    assert lib.fc_host_device_pointer(None, ctypes.byref(dev)) == fc.FC_ERR_INVALID_ARG
+    assert lib.fc_host_device_pointer(ctypes.c_void_p(A), None) == fc.FC_ERR_INVALID_ARG
     with pytest.raises(ValueError):
         fc.fc_ipc_open(b"short")
