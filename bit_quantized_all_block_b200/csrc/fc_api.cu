@@ -143,6 +143,28 @@ const FusedFnT kFusedWide[2][2][8] = {
 };
 #undef FC_WIDE7
 
+// The same for blocks whose thread group is narrower than P lanes (every lane
+// computes every rank's scale): quantized reduce-scatter step, P >= 3 (below
+// that every group is wide enough).  [dtype][w1][w2][P - 1] as kFused.
+#define FC_N3(T, B1, B2)                                                                                  \
+    {nullptr, nullptr, fc::launch_fused<T, B1, B2, 3, false, false, false>,                                \
+     fc::launch_fused<T, B1, B2, 4, false, false, false>, fc::launch_fused<T, B1, B2, 5, false, false, false>, \
+     fc::launch_fused<T, B1, B2, 6, false, false, false>, fc::launch_fused<T, B1, B2, 7, false, false, false>, \
+     fc::launch_fused<T, B1, B2, 8, false, false, false>}
+#define FC_N48(T, B1, B2)                                                                                 \
+    {nullptr, nullptr, nullptr, fc::launch_fused<T, B1, B2, 4, false, false, false>,                      \
+     nullptr, nullptr, nullptr, fc::launch_fused<T, B1, B2, 8, false, false, false>}
+#define FC_NONE {nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr}
+#define FC_DTYPE(T)                                                                               \
+    {{FC_N3(T, 4, 4), FC_N48(T, 4, 8), FC_N48(T, 4, 16)},                                        \
+     {FC_N48(T, 8, 4), FC_N3(T, 8, 8), FC_N48(T, 8, 16)},                                        \
+     {FC_NONE, FC_NONE, FC_NONE}}
+const FusedFnT kFusedNarrow[2][3][3][8] = {FC_DTYPE(__half), FC_DTYPE(__nv_bfloat16)};
+#undef FC_DTYPE
+#undef FC_NONE
+#undef FC_N48
+#undef FC_N3
+
 int width_index(int bits) { return bits == 4 ? 0 : bits == 8 ? 1 : bits == 16 ? 2 : -1; }
 
 // The fused kernel's latency shape (64-thread CTAs, 8 elements per thread) for
@@ -161,7 +183,8 @@ const FusedFnT kFusedSmall[2][2][3] = {
 
 FusedFnT small_variant(fc_dtype dtype, int bits_rs, int bits_ag, int P, int block, size_t n)
 {
-    if (bits_rs != bits_ag || bits_rs == 16 || block > 256 || n * (size_t)P > (size_t)FC_SMALL_MAX_ELEMS)
+    if (bits_rs != bits_ag || bits_rs == 16 || block > 256 || n * (size_t)P > (size_t)FC_SMALL_MAX_ELEMS ||
+        !fc::fused_lane_split(block, P, true))
         return nullptr;
     const int pi = P == 2 ? 0 : P == 4 ? 1 : P == 8 ? 2 : -1;
     return pi < 0 ? nullptr : kFusedSmall[dtype][bits_rs == 4][pi];
@@ -310,6 +333,9 @@ fc_status fc_quantized_allreduce_ex(const void* const* x, int P, fc_dtype dtype,
     FusedFnT fn = kFused[dtype][w1][w2][P - 1];
     if (fn == nullptr)
         return FC_ERR_UNSUPPORTED;
+    const bool split = w1 == 2 || fc::fused_lane_split(block, P, false);   // no scales when RS is unquantized
+    if (!split)
+        fn = kFusedNarrow[dtype][w1][w2][P - 1];
     FusedFnT small = small_variant(dtype, bits_rs, bits_ag, P, block, n);
     if (small != nullptr)
         fn = small;
@@ -346,7 +372,7 @@ fc_status fc_quantized_allreduce_ex(const void* const* x, int P, fc_dtype dtype,
     }
     if (any_overlap(outs, nout, ins, P))
         return FC_ERR_INVALID_ARG;
-    if (small == nullptr && bits_rs == bits_ag && bits_rs != 16) {
+    if (small == nullptr && split && bits_rs == bits_ag && bits_rs != 16) {
         bool wide = aligned32(y);
         for (int r = 0; r < P; r++)
             wide = wide && aligned32(x[r]);

@@ -271,8 +271,8 @@ __device__ __forceinline__ void rank_body_plain(const uint4* raw, float* acc)
 // or 16 (16 = that step sends fp16/bf16 values unquantized; Fig. 5 right of
 // the page compares quantizing before RS with quantizing before AG).
 // WIDE: inputs and output are moved with 32-byte accesses (every x[r] and y
-// 32-byte aligned; NC even).
-template <class T, int B1, int B2, int P, bool SMALL = false, bool WIDE = false>
+// 32-byte aligned; NC even).  SPLIT: see the step-1 scales below.
+template <class T, int B1, int B2, int P, bool SMALL = false, bool WIDE = false, bool SPLIT = true>
 __global__ void __launch_bounds__(FuShape<P, SMALL>::THREADS, FuShape<P, SMALL>::MIN_CTAS)
     k_fused(const FusedArgs a)
 {
@@ -289,7 +289,11 @@ __global__ void __launch_bounds__(FuShape<P, SMALL>::THREADS, FuShape<P, SMALL>:
     const int Lw = L < 32 ? L : 32;            // threads of the block inside this warp
     const int lane = threadIdx.x & 31;
     const int grp = lane & ~(Lw - 1);          // first lane of my group in the warp
-    const bool split = Lw >= P;                // lane r of the group computes rank r
+    // SPLIT: lane r of a block's group computes rank r's scale (the host
+    // selects this form only when the group has at least P lanes); otherwise
+    // every lane computes every rank's scale.  A compile-time choice keeps the
+    // unused form out of the unrolled rank loop.
+    constexpr bool split = SPLIT;
     const size_t toff = (size_t)threadIdx.x * E;
     const size_t stride = (size_t)gridDim.x * TILE;
     const float cq1 = __uint_as_float(FC_MAGIC_BITS + (uint32_t)((1 << QB1) - 1));
@@ -365,7 +369,7 @@ __global__ void __launch_bounds__(FuShape<P, SMALL>::THREADS, FuShape<P, SMALL>:
             // ---- step-1 scales: one lane per rank when the group is wide enough
             BlockQ mine;
             bool clamp1 = false;
-            if (split) {
+            if constexpr (split) {
                 const int me = lane - grp;
                 uint32_t um = u[0];
 #pragma unroll
@@ -382,7 +386,7 @@ __global__ void __launch_bounds__(FuShape<P, SMALL>::THREADS, FuShape<P, SMALL>:
             for (int r = 0; r < P; r++) {
                 BlockQ b;
                 bool clamp = clamp1;
-                if (split) {
+                if constexpr (split) {
                     b = shfl_blockq(mine, grp + r, cq1);
                 } else {
                     const T2 t = as_t2<T2>(u[r]);
@@ -390,17 +394,16 @@ __global__ void __launch_bounds__(FuShape<P, SMALL>::THREADS, FuShape<P, SMALL>:
                     b = block_q<QB1>(fminf(P2::lo(t), 0.0f), mx);
                     clamp = __any_sync(0xffffffffu, top_code_overflows(mx, b));
                 }
-                if (r == 0) {
-                    if (clamp)
-                        rank_body<T, QB1, NC, true, true>(raw[r], b, acc, store1, a.step1[r], e, leader, k);
-                    else
-                        rank_body<T, QB1, NC, false, true>(raw[r], b, acc, store1, a.step1[r], e, leader, k);
-                } else {
-                    if (clamp)
-                        rank_body<T, QB1, NC, true, false>(raw[r], b, acc, store1, a.step1[r], e, leader, k);
-                    else
-                        rank_body<T, QB1, NC, false, false>(raw[r], b, acc, store1, a.step1[r], e, leader, k);
-                }
+                // One copy of the rank body per rank (the loop is unrolled P
+                // times, so code size matters): when no block of this warp
+                // needs the upper clamp, its limit is +inf and the clamp is a
+                // no-op instead of a second copy of the body.
+                if (!clamp)
+                    b.cq = __int_as_float(0x7f800000);
+                if (r == 0)
+                    rank_body<T, QB1, NC, true, true>(raw[r], b, acc, store1, a.step1[r], e, leader, k);
+                else
+                    rank_body<T, QB1, NC, true, false>(raw[r], b, acc, store1, a.step1[r], e, leader, k);
                 if (valid_next)   // refill rank r with the next tile while this one finishes
                     load_chunks<T, NC, WIDE>(raw[r], static_cast<const T*>(a.x[r]) + e + stride);
             }

@@ -61,8 +61,19 @@ struct FusedArgs {
 template <class T, int BITS> cudaError_t launch_quantize(const QuantArgs& a, cudaStream_t st);
 template <int BITS, int P> cudaError_t launch_rs(const RsArgs& a, cudaStream_t st);
 template <class T, int BITS, bool WIDE = false> cudaError_t launch_ag(const AgArgs& a, cudaStream_t st);
-template <class T, int B1, int B2, int P, bool SMALL = false, bool WIDE = false>
+template <class T, int B1, int B2, int P, bool SMALL = false, bool WIDE = false, bool SPLIT = true>
 cudaError_t launch_fused(const FusedArgs& a, cudaStream_t st);
+
+// Elements per thread per rank of the fused kernel's bandwidth and latency
+// shapes.  A block is L = block / E threads; the lane-split scale form (SPLIT)
+// needs min(L, 32) >= P.
+constexpr int FC_FUSED_E = 16;
+constexpr int FC_FUSED_SMALL_E = 8;
+inline bool fused_lane_split(int block, int P, bool small)
+{
+    const int L = block / (small ? FC_FUSED_SMALL_E : FC_FUSED_E);
+    return (L < 32 ? L : 32) >= P;
+}
 
 // Persistent grid: enough CTAs of `threads` threads to fill every SM at the
 // kernel's occupancy, never more than there are tiles of `tile` elements.

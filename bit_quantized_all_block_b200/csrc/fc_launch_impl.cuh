@@ -38,16 +38,17 @@ cudaError_t launch_ag(const AgArgs& a, cudaStream_t st)
     return cudaGetLastError();
 }
 
-template <class T, int B1, int B2, int P, bool SMALL, bool WIDE>
+template <class T, int B1, int B2, int P, bool SMALL, bool WIDE, bool SPLIT>
 cudaError_t launch_fused(const FusedArgs& a, cudaStream_t st)
 {
     using S = FuShape<P, SMALL>;
+    static_assert(S::E == (SMALL ? FC_FUSED_SMALL_E : FC_FUSED_E), "fused_lane_split() assumes this shape");
     int grid = 0;
     cudaError_t e =
-        persistent_grid((const void*)k_fused<T, B1, B2, P, SMALL, WIDE>, S::THREADS, a.n, S::TILE, &grid);
+        persistent_grid((const void*)k_fused<T, B1, B2, P, SMALL, WIDE, SPLIT>, S::THREADS, a.n, S::TILE, &grid);
     if (e != cudaSuccess)
         return e;
-    k_fused<T, B1, B2, P, SMALL, WIDE><<<grid, S::THREADS, 0, st>>>(a);
+    k_fused<T, B1, B2, P, SMALL, WIDE, SPLIT><<<grid, S::THREADS, 0, st>>>(a);
     return cudaGetLastError();
 }
 
