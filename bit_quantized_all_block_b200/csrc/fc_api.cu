@@ -129,19 +129,17 @@ const FusedFnT kFused[2][3][3][8] = {FC_DTYPE(__half), FC_DTYPE(__nv_bfloat16)};
 #undef FC_P248
 #undef FC_ALLP
 // Equal quantized widths with 32-byte accesses of the inputs and the output,
-// for every x[r] and y 32-byte aligned: [dtype][bits == 4][P - 1].  Not for
-// INT8 at P = 8, where the wide form spills registers and is slower.
-#define FC_WIDE7(T, B)                                                                             \
-    fc::launch_fused<T, B, B, 1, false, true>, fc::launch_fused<T, B, B, 2, false, true>,            \
-        fc::launch_fused<T, B, B, 3, false, true>, fc::launch_fused<T, B, B, 4, false, true>,        \
-        fc::launch_fused<T, B, B, 5, false, true>, fc::launch_fused<T, B, B, 6, false, true>,        \
-        fc::launch_fused<T, B, B, 7, false, true>
+// for every x[r] and y 32-byte aligned: [dtype][bits == 4][P - 1].
+#define FC_WIDE(T, B)                                                                              \
+    {fc::launch_fused<T, B, B, 1, false, true>, fc::launch_fused<T, B, B, 2, false, true>,           \
+     fc::launch_fused<T, B, B, 3, false, true>, fc::launch_fused<T, B, B, 4, false, true>,           \
+     fc::launch_fused<T, B, B, 5, false, true>, fc::launch_fused<T, B, B, 6, false, true>,           \
+     fc::launch_fused<T, B, B, 7, false, true>, fc::launch_fused<T, B, B, 8, false, true>}
 const FusedFnT kFusedWide[2][2][8] = {
-    {{FC_WIDE7(__half, 8), nullptr}, {FC_WIDE7(__half, 4), fc::launch_fused<__half, 4, 4, 8, false, true>}},
-    {{FC_WIDE7(__nv_bfloat16, 8), nullptr},
-     {FC_WIDE7(__nv_bfloat16, 4), fc::launch_fused<__nv_bfloat16, 4, 4, 8, false, true>}},
+    {FC_WIDE(__half, 8), FC_WIDE(__half, 4)},
+    {FC_WIDE(__nv_bfloat16, 8), FC_WIDE(__nv_bfloat16, 4)},
 };
-#undef FC_WIDE7
+#undef FC_WIDE
 
 // The same for blocks whose thread group is narrower than P lanes (every lane
 // computes every rank's scale): quantized reduce-scatter step, P >= 3 (below
@@ -376,7 +374,7 @@ fc_status fc_quantized_allreduce_ex(const void* const* x, int P, fc_dtype dtype,
         bool wide = aligned32(y);
         for (int r = 0; r < P; r++)
             wide = wide && aligned32(x[r]);
-        if (wide && kFusedWide[dtype][bits_rs == 4][P - 1] != nullptr)
+        if (wide)
             fn = kFusedWide[dtype][bits_rs == 4][P - 1];
     }
     fc::FusedArgs a{};

@@ -20,9 +20,14 @@
 //  * the P per-rank scale computations of a block are spread over the lanes
 //    of its group (lane r computes rank r) and broadcast with shuffles;
 //  * the upper code clamp binds only when the block maximum's code rounds to
-//    qmax + 1 -- rare -- so it is checked once per block from the maximum and
-//    applied through a warp-uniform branch; the lower clamp never binds
-//    (see the lower-clamp note in fc_device.cuh);
+//    qmax + 1 -- rare -- so it is checked once per block from the maximum;
+//    when no block of the warp needs it, its limit is +inf, so one copy of
+//    each body serves both cases (the rank loop is unrolled P times and its
+//    code size shows up as instruction-fetch stalls); the lower clamp never
+//    binds (see the lower-clamp note in fc_device.cuh);
+//  * the P per-rank scale computations use the lane-split form whenever a
+//    block's thread group has at least P lanes (SPLIT, chosen by the host
+//    from the block size), so the unrolled loop carries only one form;
 //  * each rank's registers are refilled with the next tile's data as soon as
 //    that rank is consumed, so loads stay in flight during the rest of the
 //    tile (software pipelining without extra registers);
@@ -138,13 +143,13 @@ __device__ __forceinline__ void store_thread_codes(uint8_t* codes, size_t e, con
 
 // Step-1 work on one rank's values, chunk by chunk: quantize, dequantize,
 // accumulate in rank order; optionally store codes, scale and zero-point.
-template <class T, int BITS, int NC, bool CLAMP, bool FIRST>
+template <class T, int BITS, int NC, bool FIRST>
 __device__ __forceinline__ void rank_body(const uint4* raw, const BlockQ& b, float* acc, bool store,
                                           const QPtr& out, size_t e, bool leader, size_t k)
 {
     using P2 = Pair<T>;
     using T2 = typename P2::T2;
-    const float cqz = __fsub_rn(b.cq, b.zf);   // FC_MAGIC + qmax - z (exact)
+    const float cqz = __fsub_rn(b.cq, b.zf);   // FC_MAGIC + qmax - z (exact; +inf: no clamp)
     uint32_t words[NC * BITS / 4];
 #pragma unroll
     for (int c = 0; c < NC; c++) {
@@ -158,8 +163,7 @@ __device__ __forceinline__ void rank_body(const uint4* raw, const BlockQ& b, flo
         }
 #pragma unroll
         for (int i = 0; i < 8; i++) {
-            if (CLAMP)
-                r[i] = fminf(r[i], cqz);
+            r[i] = fminf(r[i], cqz);
             const float xh = __fmul_rn(__fsub_rn(r[i], FC_MAGIC), b.s);  // (q - z) * s
             acc[c * 8 + i] = FIRST ? xh : __fadd_rn(acc[c * 8 + i], xh);
         }
@@ -181,7 +185,7 @@ __device__ __forceinline__ void rank_body(const uint4* raw, const BlockQ& b, flo
 }
 
 // Step 2 on the sums, chunk by chunk: requantize, dequantize, store y (+ payload).
-template <class T, int BITS, int NC, bool CLAMP, bool WIDE>
+template <class T, int BITS, int NC, bool WIDE>
 __device__ __forceinline__ void sum_body(const float* acc, const BlockQ& b, T* y, bool store,
                                          const QPtr& out, size_t e, bool leader, size_t k)
 {
@@ -194,8 +198,7 @@ __device__ __forceinline__ void sum_body(const float* acc, const BlockQ& b, T* y
 #pragma unroll
         for (int i = 0; i < 8; i++) {
             r[i] = round_product_shifted(acc[c * 8 + i], b.inv);
-            if (CLAMP)
-                r[i] = fminf(r[i], cqz);
+            r[i] = fminf(r[i], cqz);
             o[i] = __fmul_rn(__fsub_rn(r[i], FC_MAGIC), b.s);
         }
         if constexpr (WIDE)
@@ -401,9 +404,9 @@ __global__ void __launch_bounds__(FuShape<P, SMALL>::THREADS, FuShape<P, SMALL>:
                 if (!clamp)
                     b.cq = __int_as_float(0x7f800000);
                 if (r == 0)
-                    rank_body<T, QB1, NC, true, true>(raw[r], b, acc, store1, a.step1[r], e, leader, k);
+                    rank_body<T, QB1, NC, true>(raw[r], b, acc, store1, a.step1[r], e, leader, k);
                 else
-                    rank_body<T, QB1, NC, true, false>(raw[r], b, acc, store1, a.step1[r], e, leader, k);
+                    rank_body<T, QB1, NC, false>(raw[r], b, acc, store1, a.step1[r], e, leader, k);
                 if (valid_next)   // refill rank r with the next tile while this one finishes
                     load_chunks<T, NC, WIDE>(raw[r], static_cast<const T*>(a.x[r]) + e + stride);
             }
@@ -431,15 +434,12 @@ __global__ void __launch_bounds__(FuShape<P, SMALL>::THREADS, FuShape<P, SMALL>:
             mx = fmaxf(mx, acc[E - 1]);
             // the next tile's step-1 barrier separates these reads from the next writes
             group_minmax_f32<B1 == 16>(mn, mx, L, red32);
-            const BlockQ b2 = block_q<B2>(mn, mx);
+            BlockQ b2 = block_q<B2>(mn, mx);
             const bool clamp2 = __any_sync(0xffffffffu, top_code_overflows(mx, b2));
-            if (valid) {
-                const bool store2 = a.write_step2 != 0;
-                if (clamp2)
-                    sum_body<T, B2, NC, true, WIDE>(acc, b2, y, store2, a.step2, e, leader, k);
-                else
-                    sum_body<T, B2, NC, false, WIDE>(acc, b2, y, store2, a.step2, e, leader, k);
-            }
+            if (!clamp2)
+                b2.cq = __int_as_float(0x7f800000);   // one body: the clamp is a no-op
+            if (valid)
+                sum_body<T, B2, NC, WIDE>(acc, b2, y, a.write_step2 != 0, a.step2, e, leader, k);
         }
     }
 }

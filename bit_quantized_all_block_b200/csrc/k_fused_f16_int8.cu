@@ -1,5 +1,5 @@
-// Instantiations of the fused all-reduce kernel: __half, INT8 in both steps, P = 1..8 with
-// 16-byte global accesses, P = 1..7 also with 32-byte ones.
+// Instantiations of the fused all-reduce kernel: __half, INT8 in both steps, P = 1..8, with
+// 16-byte and with 32-byte global accesses.
 #include "fc_launch_impl.cuh"
 
 namespace fc {
@@ -18,4 +18,5 @@ template cudaError_t launch_fused<__half, 8, 8, 4, false, true>(const FusedArgs&
 template cudaError_t launch_fused<__half, 8, 8, 5, false, true>(const FusedArgs&, cudaStream_t);
 template cudaError_t launch_fused<__half, 8, 8, 6, false, true>(const FusedArgs&, cudaStream_t);
 template cudaError_t launch_fused<__half, 8, 8, 7, false, true>(const FusedArgs&, cudaStream_t);
+template cudaError_t launch_fused<__half, 8, 8, 8, false, true>(const FusedArgs&, cudaStream_t);
 }  // namespace fc
