@@ -348,41 +348,43 @@ __global__ void __launch_bounds__(FuShape<P, SMALL>::THREADS, FuShape<P, SMALL>:
                 for (int r = 0; r < P; r++)
                     u[r] = t2_bits(__hmin2(as_t2<T2>(u[r]), as_t2<T2>(__shfl_xor_sync(0xffffffffu, u[r], o))));
             }
-            if (L > 32) {                       // blocks that span warps
-                if (lane == 0) {
-#pragma unroll
-                    for (int r = 0; r < P; r++)
-                        red16[r][threadIdx.x >> 5] = u[r];
-                }
-                __syncthreads();
-                const int nw = L >> 5, w0 = (threadIdx.x / L) * nw;
-#pragma unroll
-                for (int r = 0; r < P; r++) {
-                    uint32_t v = red16[r][w0];
-                    for (int i = 1; i < nw; i++)
-                        v = t2_bits(__hmin2(as_t2<T2>(v), as_t2<T2>(red16[r][w0 + i])));
-                    u[r] = v;
-                }
-                // With both steps quantized, the step-2 reduction's barrier
-                // separates these reads from the next tile's writes.
-                if (B2 == 16)
-                    __syncthreads();
-            }
-
             // ---- step-1 scales: one lane per rank when the group is wide enough
             BlockQ mine;
             bool clamp1 = false;
             if constexpr (split) {
+                // lane `me` of the group computes rank me's scale (lanes past
+                // P duplicate rank 0); it needs only that rank's extremes
                 const int me = lane - grp;
-                uint32_t um = u[0];
+                const int rr = me < P ? me : 0;
+                uint32_t um;
+                if (L > 32) {                   // blocks that span warps
+                    if (lane == 0) {
 #pragma unroll
-                for (int r = 1; r < P; r++)
-                    um = (me == r) ? u[r] : um;
+                        for (int r = 0; r < P; r++)
+                            red16[r][threadIdx.x >> 5] = u[r];
+                    }
+                    __syncthreads();
+                    const int nw = L >> 5, w0 = (threadIdx.x / L) * nw;
+                    um = red16[rr][w0];
+                    for (int i = 1; i < nw; i++)
+                        um = t2_bits(__hmin2(as_t2<T2>(um), as_t2<T2>(red16[rr][w0 + i])));
+                    // With both steps quantized, the step-2 reduction's barrier
+                    // separates these reads from the next tile's writes.
+                    if (B2 == 16)
+                        __syncthreads();
+                } else {
+                    um = u[0];
+#pragma unroll
+                    for (int r = 1; r < P; r++)
+                        um = (rr == r) ? u[r] : um;
+                }
                 const T2 t = as_t2<T2>(um);
                 const float mx = fmaxf(-P2::hi(t), 0.0f);
                 mine = block_q<QB1>(fminf(P2::lo(t), 0.0f), mx);
                 clamp1 = __any_sync(0xffffffffu, top_code_overflows(mx, mine));
             }
+            // (without SPLIT the group is narrower than P lanes, so L < 32 and
+            // every lane holds every rank's extremes in u)
 
             const bool store1 = a.write_step1 && valid;
 #pragma unroll
