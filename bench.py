@@ -71,11 +71,20 @@ def algorithmic_bytes(w, variant: str) -> int:
     raise ValueError(variant)
 
 
+def _code_only(text: str) -> str:
+    """C++ source with comments removed and whitespace collapsed (comment edits
+    do not change the compiled kernel, so they keep the recorded traffic valid)."""
+    import re
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
 def source_hash() -> str:
     h = hashlib.sha256()
     for p in KERNEL_SOURCES:
         h.update(os.path.basename(p).encode())
-        h.update(open(p, "rb").read())
+        h.update(_code_only(open(p).read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -10,13 +10,12 @@
 // The kernel moves ~1 GB per call on the 70B-shaped workload and runs close to
 // both the HBM and the instruction-issue ceilings (about a dozen operations per
 // input element), so it is laid out to cut instructions:
-//  * thread t of a CTA owns E contiguous elements of every rank in the tile
-//    (E = 32 for P <= 4, 16 above, to stay in registers); a block of B elements
-//    is L = B/E consecutive threads, so a 128-block needs 4 threads and 2
-//    shuffle rounds.  All loads and stores of a thread use one base pointer
-//    with immediate offsets; codes leave as 128-bit stores.  Loads go through
-//    L1 because the two halves of each 32-byte sector are read by consecutive
-//    instructions of the same thread;
+//  * thread t of a CTA owns E = 16 contiguous elements of every rank in the
+//    tile (8 in the latency shape); a block of B elements is L = B/E
+//    consecutive threads, so a 128-block needs 8 threads and 3 shuffle
+//    rounds.  All loads and stores of a thread use one base pointer with
+//    immediate offsets; a thread's 32 bytes of a rank move as one 32-byte
+//    access when the buffers allow it (WIDE), else as two 16-byte ones;
 //  * the P per-rank scale computations of a block are spread over the lanes
 //    of its group (lane r computes rank r) and broadcast with shuffles;
 //  * the upper code clamp binds only when the block maximum's code rounds to
@@ -25,9 +24,10 @@
 //    each body serves both cases (the rank loop is unrolled P times and its
 //    code size shows up as instruction-fetch stalls); the lower clamp never
 //    binds (see the lower-clamp note in fc_device.cuh);
-//  * the P per-rank scale computations use the lane-split form whenever a
-//    block's thread group has at least P lanes (SPLIT, chosen by the host
-//    from the block size), so the unrolled loop carries only one form;
+//    that lane-split form is used whenever a block's thread group has at
+//    least P lanes (SPLIT, chosen by the host from the block size; narrower
+//    groups compute every rank's scale in every lane), so the unrolled loop
+//    carries only one form;
 //  * each rank's registers are refilled with the next tile's data as soon as
 //    that rank is consumed, so loads stay in flight during the rest of the
 //    tile (software pipelining without extra registers);
