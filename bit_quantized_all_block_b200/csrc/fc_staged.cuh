@@ -80,6 +80,8 @@ __device__ __forceinline__ void chunk_shifted(const uint32_t* w, int c, float* s
 }
 
 // Block extremes (0 folded in) of E fp32 values held by each of L threads.
+// `red` alternates between two halves from tile to tile, so one barrier per
+// tile separates every write from the reads of the previous use of its half.
 template <int E>
 __device__ __forceinline__ void block_minmax_f32(const float* v, int L, float2* red, float& mn, float& mx)
 {
@@ -92,7 +94,7 @@ __device__ __forceinline__ void block_minmax_f32(const float* v, int L, float2* 
     }
     mn = fminf(mn, v[E - 1]);
     mx = fmaxf(mx, v[E - 1]);
-    group_minmax_f32(mn, mx, L, red);
+    group_minmax_f32<false>(mn, mx, L, red);
 }
 
 // Quantize E fp32 values (one thread's share of a block) and store codes,
@@ -130,7 +132,7 @@ __global__ void __launch_bounds__(ST_THREADS) k_quantize(const QuantArgs a)
     using P2 = Pair<T>;
     using T2 = typename P2::T2;
     constexpr int NC = QuantShape::NC, E = QuantShape::E, TILE = QuantShape::TILE;
-    __shared__ uint32_t red[ST_THREADS / 32];
+    __shared__ uint32_t red[2][ST_THREADS / 32];   // alternating halves: one barrier per tile
     const int L = a.block / E;
     const int j = threadIdx.x % L;
     const int lg_block = __ffs(a.block) - 1;
@@ -149,11 +151,12 @@ __global__ void __launch_bounds__(ST_THREADS) k_quantize(const QuantArgs a)
                 raw[c] = make_uint4(0, 0, 0, 0);
         }
     }
-    for (size_t base = (size_t)blockIdx.x * TILE; base < a.n; base += stride) {
+    int half = 0;
+    for (size_t base = (size_t)blockIdx.x * TILE; base < a.n; base += stride, half ^= 1) {
         const size_t e = base + toff;
         const bool valid = e < a.n;
         const size_t k = e >> lg_block;
-        const T2 t = as_t2<T2>(group_min_negmax<T>(local_min_negmax<T, NC>(raw), L, red));
+        const T2 t = as_t2<T2>(group_min_negmax<T, false>(local_min_negmax<T, NC>(raw), L, red[half]));
         const float mx = fmaxf(-P2::hi(t), 0.0f);
         const BlockQ b = block_q<BITS>(fminf(P2::lo(t), 0.0f), mx);
         const bool clamp = __any_sync(0xffffffffu, top_code_overflows(mx, b));
@@ -188,7 +191,7 @@ __global__ void __launch_bounds__(ST_THREADS) k_rs(const RsArgs a)
 {
     constexpr int NC = RsShape<P>::NC, E = RsShape<P>::E, TILE = RsShape<P>::TILE;
     constexpr int NW = NC * BITS / 4;
-    __shared__ float2 red[ST_THREADS / 32];
+    __shared__ float2 red[2][ST_THREADS / 32];     // alternating halves: one barrier per tile
     const int L = a.block / E;
     const int j = threadIdx.x % L;
     const int lg_block = __ffs(a.block) - 1;
@@ -215,7 +218,8 @@ __global__ void __launch_bounds__(ST_THREADS) k_rs(const RsArgs a)
             }
         }
     }
-    for (size_t base = (size_t)blockIdx.x * TILE; base < a.n; base += stride) {
+    int half = 0;
+    for (size_t base = (size_t)blockIdx.x * TILE; base < a.n; base += stride, half ^= 1) {
         const size_t e = base + toff;
         const bool valid = e < a.n;
         const bool valid_next = e + stride < a.n;
@@ -241,7 +245,7 @@ __global__ void __launch_bounds__(ST_THREADS) k_rs(const RsArgs a)
             }
         }
         float mn, mx;
-        block_minmax_f32<E>(acc, L, red, mn, mx);
+        block_minmax_f32<E>(acc, L, red[half], mn, mx);
         const BlockQ b = block_q<BITS>(mn, mx);
         const bool clamp = __any_sync(0xffffffffu, top_code_overflows(mx, b));
         if (valid) {
