@@ -111,19 +111,6 @@ __device__ __forceinline__ bool top_code_overflows(float mx, const BlockQ& b)
     return __fadd_rn(round_product_shifted(mx, b.inv), b.zf) > b.cq;
 }
 
-// Pack the 8 shifted codes of one chunk into the thread's code words:
-// INT8 -> words[2c], words[2c+1]; INT4 -> words[c].
-template <int BITS>
-__device__ __forceinline__ void pack_chunk(const float* sh, uint32_t* words, int c)
-{
-    if constexpr (BITS == 8) {
-        words[2 * c] = pack4_u8(sh);
-        words[2 * c + 1] = pack4_u8(sh + 4);
-    } else {
-        words[c] = pack8_u4(sh);
-    }
-}
-
 // Store a thread's E codes (E*BITS/8 contiguous bytes) at element offset e.
 template <int BITS, int NC>
 __device__ __forceinline__ void store_thread_codes(uint8_t* codes, size_t e, const uint32_t* w)
@@ -167,13 +154,8 @@ __device__ __forceinline__ void rank_body(const uint4* raw, const BlockQ& b, flo
             const float xh = __fmul_rn(__fsub_rn(r[i], FC_MAGIC), b.s);  // (q - z) * s
             acc[c * 8 + i] = FIRST ? xh : __fadd_rn(acc[c * 8 + i], xh);
         }
-        if (store) {
-            float sh[8];
-#pragma unroll
-            for (int i = 0; i < 8; i++)
-                sh[i] = __fadd_rn(r[i], b.zf);                            // FC_MAGIC + q
-            pack_chunk<BITS>(sh, words, c);
-        }
+        if (store)
+            pack_shifted<BITS>(r, b, pack_offset<BITS>(b), words, c);
     }
     if (store) {
         store_thread_codes<BITS, NC>(out.codes, e, words);
@@ -205,13 +187,8 @@ __device__ __forceinline__ void sum_body(const float* acc, const BlockQ& b, T* y
             ov[c] = narrow8<T>(o);
         else
             st_stream(y + e + c * FC_CHUNK, narrow8<T>(o));
-        if (store) {
-            float sh[8];
-#pragma unroll
-            for (int i = 0; i < 8; i++)
-                sh[i] = __fadd_rn(r[i], b.zf);
-            pack_chunk<BITS>(sh, words, c);
-        }
+        if (store)
+            pack_shifted<BITS>(r, b, pack_offset<BITS>(b), words, c);
     }
     if constexpr (WIDE)
         store_chunks<NC, true>(y + e, ov);

@@ -249,17 +249,18 @@ __device__ __forceinline__ void epilogue_block(uint32_t taddr, const GemmQuantAr
     const float mx = fmaxf(fmaxf(P2::lo(M), P2::hi(M)), 0.0f);
     const BlockQ b = block_q<BITS>(mn, mx);
     const float cqz = __fsub_rn(b.cq, b.zf);
+    const uint32_t offset = pack_offset<BITS>(b);
     uint32_t words[NB * BITS / 32];
 #pragma unroll
     for (int c = 0; c < NB / 8; c++) {
-        float sh[8];
+        float r[8];
 #pragma unroll
         for (int h = 0; h < 4; h++) {
             const float2 f = P2::to_f2(as_t2<T2>(v16[c * 4 + h]));
-            sh[2 * h] = __fadd_rn(fminf(round_product_shifted(f.x, b.inv), cqz), b.zf);
-            sh[2 * h + 1] = __fadd_rn(fminf(round_product_shifted(f.y, b.inv), cqz), b.zf);
+            r[2 * h] = fminf(round_product_shifted(f.x, b.inv), cqz);
+            r[2 * h + 1] = fminf(round_product_shifted(f.y, b.inv), cqz);
         }
-        pack_chunk<BITS>(sh, words, c);
+        pack_shifted<BITS>(r, b, offset, words, c);
     }
     const size_t e = row * (size_t)a.N + col;     // flat element index of the block
     uint4* cdst = reinterpret_cast<uint4*>(a.out.codes + e * BITS / 8);

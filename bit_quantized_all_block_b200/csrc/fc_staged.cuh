@@ -104,18 +104,18 @@ __device__ __forceinline__ void quant_store(const float* v, const BlockQ& b, con
                                             bool leader, size_t k)
 {
     const float cqz = __fsub_rn(b.cq, b.zf);
+    const uint32_t offset = pack_offset<BITS>(b);
     uint32_t words[NC * BITS / 4];
 #pragma unroll
     for (int c = 0; c < NC; c++) {
-        float sh[8];
+        float r[8];
 #pragma unroll
         for (int i = 0; i < 8; i++) {
-            float r = round_product_shifted(v[c * 8 + i], b.inv);
+            r[i] = round_product_shifted(v[c * 8 + i], b.inv);
             if (CLAMP)
-                r = fminf(r, cqz);
-            sh[i] = __fadd_rn(r, b.zf);
+                r[i] = fminf(r[i], cqz);
         }
-        pack_chunk<BITS>(sh, words, c);
+        pack_shifted<BITS>(r, b, offset, words, c);
     }
     store_thread_codes<BITS, NC>(out.codes, e, words);
     if (leader) {
