@@ -1,8 +1,8 @@
 """Full-size GPU parity: the fused all-reduce runs on the whole workload (the
-launch bench.py times, payloads written), then sampled token rows -- first,
-last and seeded random rows -- are checked bit for bit against the oracle run
-on exactly those rows (every block depends only on the same block of every
-rank, so a row sample is an independent all-reduce).  The staged pipeline is
+launch bench.py times, payloads written) and its whole output and every
+payload are checked bit for bit against the CPU oracle run over every token
+row (on all host cores: every block depends only on the same block of every
+rank, so row slices are independent all-reduces).  The staged pipeline is
 compared with the fused kernel on the whole output."""
 import functools
 
@@ -11,9 +11,9 @@ import pytest
 import torch
 
 import bit_quantized_all_block_b200 as fc
-import oracle
 from bit_quantized_all_block_b200 import synth
 from tests.gpu_util import to_dev
+from tests.oracle_rows import allreduce_all_rows
 
 pytestmark = pytest.mark.gpu
 
@@ -25,18 +25,8 @@ def inputs(P, T, H, dtype, frac, factor, seed):
     return synth.partials(P, T, H, dtype, frac, factor, seed)
 
 
-def sample_rows(T, k=16, seed=0):
-    rng = np.random.default_rng(seed)
-    mid = rng.choice(np.arange(8, T - 8), size=k, replace=False)
-    return np.sort(np.concatenate([np.arange(8), mid, np.arange(T - 8, T)]))
-
-
-def rows_of(a, rows, width):
-    return a.reshape(-1, width)[rows].ravel()
-
-
 @pytest.mark.parametrize("w", FULL, ids=lambda w: w.name)
-def test_full_size_sampled_rows(w):
+def test_full_size_every_output(w):
     xs = inputs(w.P, w.T, w.H, w.dtype, w.outlier_frac, w.outlier_factor, w.seed)
     xd = to_dev(xs, w.dtype)
     s1 = [fc.QBuf.empty(w.n, w.bits, w.block) for _ in range(w.P)]
@@ -44,20 +34,14 @@ def test_full_size_sampled_rows(w):
     y = fc.fc_quantized_allreduce(xd, w.bits, w.block, step1=s1, step2=s2)
     torch.cuda.synchronize()
 
-    rows = sample_rows(w.T, seed=w.block)
-    sub = [rows_of(x, rows, w.H) for x in xs]
-    y_ref, p1_ref, p2_ref = oracle.allreduce(sub, w.dtype, w.bits, w.block)
-    idx = torch.from_numpy(rows).cuda()
-    y_rows = y.view(w.T, w.H)[idx].contiguous().view(torch.int16).cpu().numpy().view(np.uint16).ravel()
-    assert np.array_equal(y_rows, y_ref)
-
-    cb_row = w.H * w.bits // 8            # code bytes per token row
-    nb_row = w.H // w.block               # blocks per token row
-    for q, p in zip(s1 + [s2], p1_ref + [p2_ref]):
-        assert np.array_equal(q.codes.view(w.T, cb_row)[idx].cpu().numpy().ravel(), p.codes)
-        assert np.array_equal(q.scales.view(w.T, nb_row)[idx].cpu().numpy().ravel().view(np.uint32),
-                              p.scales.view(np.uint32))
-        assert np.array_equal(q.zps.view(w.T, nb_row)[idx].cpu().numpy().ravel(), p.zps)
+    y_ref, p1_ref, p2_ref = allreduce_all_rows(xs, w.T, w.H, w.dtype, w.bits, w.block)
+    got = y.view(torch.int16).cpu().numpy().view(np.uint16)
+    bad = np.nonzero(got != y_ref)[0]
+    assert bad.size == 0, f"{bad.size} of {got.size} outputs differ, first at {bad[:8]}"
+    for q, (codes, scales, zps) in zip(s1 + [s2], p1_ref + [p2_ref]):
+        assert np.array_equal(q.codes.cpu().numpy(), codes)
+        assert np.array_equal(q.scales.cpu().numpy().view(np.uint32), scales.view(np.uint32))
+        assert np.array_equal(q.zps.cpu().numpy(), zps)
 
     # staged pipeline == fused kernel on the whole tensor
     q1 = [fc.fc_quantize(x, w.bits, w.block) for x in xd]
@@ -74,15 +58,11 @@ def test_full_size_sampled_rows(w):
 @pytest.mark.parametrize("bits", [8, 4])
 @pytest.mark.parametrize("lg", [13, 16, 20, 24])
 def test_message_sweep_points(bits, lg):
-    """Decode-regime message sizes (2^lg fp16 elements per rank, P=4) in full."""
+    """Message sizes of the sweep (2^lg fp16 elements per rank, P=4) in full."""
     w = [v for v in synth.message_sweep(bits) if v.n == 1 << lg][0]
     xs = synth.workload_partials(w)
-    rows = np.arange(w.T) if w.T <= 64 else sample_rows(w.T, seed=lg)
     xd = to_dev(xs, w.dtype)
     y = fc.fc_quantized_allreduce(xd, w.bits, w.block)
     torch.cuda.synchronize()
-    sub = [rows_of(x, rows, w.H) for x in xs]
-    y_ref, _, _ = oracle.allreduce(sub, w.dtype, w.bits, w.block)
-    idx = torch.from_numpy(rows).cuda()
-    y_rows = y.view(w.T, w.H)[idx].contiguous().view(torch.int16).cpu().numpy().view(np.uint16).ravel()
-    assert np.array_equal(y_rows, y_ref)
+    y_ref, _, _ = allreduce_all_rows(xs, w.T, w.H, w.dtype, w.bits, w.block)
+    assert np.array_equal(y.view(torch.int16).cpu().numpy().view(np.uint16), y_ref)
