@@ -213,6 +213,16 @@ def _oracle_team_worker(idx, xs_slice, dtype, bits, block, runs, barrier, out_q)
         out_q.put((idx, k, t0, t1, y if k == runs - 1 else None))
 
 
+def cpu_model() -> str:
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def host_cores() -> int:
     try:
         return len(os.sched_getaffinity(0))
@@ -286,7 +296,7 @@ def run_reference(args, w):
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {"workload": w.name, "description": w.describe(), "sample": sample},
         "cpu_baseline": {"value": round(value, 6), "unit": "GB/s", "cores": procs, "kind": "oracle",
-                         "sample": sample},
+                         "sample": sample, "cpu": cpu_model()},
         "e2e": {"value": round(value, 6), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -738,7 +748,8 @@ def main():
                 one = sum(x.size for x in sub) * 2 / dt / 1e9
                 line["cpu_baseline"] = {
                     "value": round(one, 5), "unit": "GB/s", "cores": 1, "kind": "oracle",
-                    "sample": f"{rows} of {w.T} token rows per rank, {dt:.1f} s, single thread"}
+                    "sample": f"{rows} of {w.T} token rows per rank, {dt:.1f} s, single thread",
+                    "cpu": cpu_model()}
                 exact = bool(np.array_equal(y_np[: rows * w.H], y_ref))
                 try:   # the same oracle on every host core
                     times, y_team, procs = oracle_team(w, np.stack(sub), rows, 3, host_cores())
@@ -746,7 +757,7 @@ def main():
                         dt_team = min(times[1:])
                         line["cpu_baseline"] = {
                             "value": round(sum(x.size for x in sub) * 2 / dt_team / 1e9, 5), "unit": "GB/s",
-                            "cores": procs, "kind": "oracle",
+                            "cores": procs, "kind": "oracle", "cpu": cpu_model(),
                             "sample": (f"{rows} of {w.T} token rows per rank split over {procs} processes "
                                        f"(one per host core), best of 2 runs after 1 warm-up, "
                                        f"{dt_team * 1e3:.1f} ms per run"),
