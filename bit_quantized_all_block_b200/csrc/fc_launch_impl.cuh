@@ -20,7 +20,7 @@ template <int BITS, int P>
 cudaError_t launch_rs(const RsArgs& a, cudaStream_t st)
 {
     int grid = 0;
-    cudaError_t e = persistent_grid((const void*)k_rs<BITS, P>, ST_THREADS, a.n, RsShape<P>::TILE, &grid);
+    cudaError_t e = persistent_grid((const void*)k_rs<BITS, P>, ST_THREADS, a.n, RsShape<BITS, P>::TILE, &grid);
     if (e != cudaSuccess)
         return e;
     k_rs<BITS, P><<<grid, ST_THREADS, 0, st>>>(a);

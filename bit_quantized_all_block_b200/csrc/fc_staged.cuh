@@ -30,7 +30,10 @@ struct StShape {
 };
 using QuantShape = StShape<4>;                          // 32 elements per thread
 using AgShape = StShape<4>;
-template <int P> using RsShape = StShape<(P <= 4 ? 4 : 2)>;
+// Reduce-scatter: 32 elements per thread and rank, except INT8 with more than
+// four ranks (16), where 32 would hold 8 ranks x 8 code words in registers and
+// cut the occupancy.
+template <int BITS, int P> using RsShape = StShape<(BITS == 4 || P <= 4) ? 4 : 2>;
 
 // Load a thread's E codes (E*BITS/8 contiguous bytes) at element offset e;
 // WIDE: 32 bytes per load where there are 32 (codes 32-byte aligned).
@@ -189,7 +192,7 @@ __global__ void __launch_bounds__(ST_THREADS) k_quantize(const QuantArgs a)
 template <int BITS, int P>
 __global__ void __launch_bounds__(ST_THREADS) k_rs(const RsArgs a)
 {
-    constexpr int NC = RsShape<P>::NC, E = RsShape<P>::E, TILE = RsShape<P>::TILE;
+    constexpr int NC = RsShape<BITS, P>::NC, E = RsShape<BITS, P>::E, TILE = RsShape<BITS, P>::TILE;
     constexpr int NW = NC * BITS / 4;
     __shared__ float2 red[2][ST_THREADS / 32];     // alternating halves: one barrier per tile
     const int L = a.block / E;
