@@ -25,7 +25,6 @@ from __future__ import annotations
 import argparse
 import datetime
 import hashlib
-import glob
 import json
 import os
 import statistics

@@ -2,7 +2,6 @@
 Fig. 5 right): every combination of reduce-scatter and all-gather widths in
 {4, 8, 16} against the oracle's fco_allreduce_ex, bit for bit, including the
 payloads of the quantized steps."""
-import numpy as np
 import pytest
 import torch
 
