@@ -489,6 +489,72 @@ def run_latency_sweep(args):
             del g
 
 
+def run_message_sweep(args):
+    """The whole message sweep of the decode-to-prefill range: 16 KB .. 1 GB of
+    fp16 per rank (2^13 .. 2^29 elements, P=4, INT8 and INT4, blocks of 128),
+    the fused all-reduce with both payloads written.  Per size: back to back in
+    a CUDA graph of 20 calls (L2 warm for the small sizes; beyond 32 MB per rank
+    every call streams from HBM) and one call at a time after an L2 flush (cold,
+    median).  Inputs are drawn on the device from a seeded generator with the
+    synthetic recipe's shape (N(0,1) times per-channel log-normal scales); the
+    largest point holds about 7.6 GB on the device."""
+    import torch
+
+    import bit_quantized_all_block_b200 as fc
+
+    torch.cuda.set_device(0)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    peak, peak_kind = read_peak()
+    gen = torch.Generator(device="cuda")
+    for bits in (8, 4):
+        for w in synth.message_sweep(bits):
+            gen.manual_seed(1000 + w.T)
+            scale = torch.exp(torch.randn(w.H, device="cuda", generator=gen) * 0.5)
+            xs = [(torch.randn(w.T, w.H, device="cuda", generator=gen) * scale).half().reshape(-1)
+                  for _ in range(w.P)]
+            y = torch.empty(w.n, dtype=torch.float16, device="cuda")
+            s1 = [fc.QBuf.empty(w.n, bits, w.block) for _ in range(w.P)]
+            s2 = fc.QBuf.empty(w.n, bits, w.block)
+
+            def step():
+                fc.fc_quantized_allreduce(xs, bits, w.block, y=y, step1=s1, step2=s2)
+
+            for _ in range(max(args.warmup, 3)):
+                step()
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                for _ in range(20):
+                    step()
+            g.replay()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            g.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            hot = e0.elapsed_time(e1) * 1e3 / 20
+            pairs = []
+            for _ in range(args.steps):
+                flush.zero_()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record()
+                step()
+                b.record()
+                pairs.append((a, b))
+            torch.cuda.synchronize()
+            cold = sorted(a.elapsed_time(b) * 1e3 for a, b in pairs)[len(pairs) // 2]
+            alg = algorithmic_bytes(w, "fused")
+            print(json.dumps({"mode": "message_sweep", "workload": w.name, "bytes_per_rank": 2 * w.n,
+                              "bits": bits, "us_back_to_back": round(hot, 2), "us_cold_l2_median": round(cold, 2),
+                              "input_gbs_back_to_back": round(w.P * w.n * 2 / hot / 1e3, 1),
+                              "achieved_gbs_back_to_back": round(alg / hot / 1e3, 1),
+                              "frac_back_to_back": round(alg / hot / 1e3 / peak, 4), "peak_kind": peak_kind}),
+                  flush=True)
+            del g, xs, y, s1, s2
+            torch.cuda.empty_cache()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -512,6 +578,8 @@ def main():
     ap.add_argument("--gemm-ranks", type=int, default=4, help="ranks of the tensor-parallel layer comparison")
     ap.add_argument("--latency-sweep", action="store_true",
                     help="decode regime: per-call latency over the 16 KB .. 8 MB per rank message sweep")
+    ap.add_argument("--message-sweep", action="store_true",
+                    help="the fused all-reduce over 16 KB .. 1 GB per rank (P=4, INT8 and INT4), one line each")
     ap.add_argument("--precision-sweep", action="store_true",
                     help="time the fused kernel for every (RS bits, AG bits) in {4,8,16}^2 on the "
                          "workload and report each variant's MSE (one JSON line per variant)")
@@ -528,6 +596,8 @@ def main():
         return run_gemm(args)
     if args.latency_sweep:
         return run_latency_sweep(args)
+    if args.message_sweep:
+        return run_message_sweep(args)
 
     import torch
     import torch.distributed as dist
