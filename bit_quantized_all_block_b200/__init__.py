@@ -71,6 +71,11 @@ def _lib():
         for f in ("fc_payload_sizes", "fc_quantize", "fc_rs_dequant_sum_requant", "fc_ag_dequant",
                   "fc_quantized_allreduce", "fc_quantized_allreduce_ex", "fc_gemm_quantize"):
             getattr(L, f).restype = I
+        PP = ctypes.POINTER(P)
+        L.fc_p2p_allreduce.argtypes = [I, I, I, S, I, I, P, P, QP, QP, PP, PP, ctypes.c_uint, P, I, P]
+        L.fc_p2p_allreduce_emulated.argtypes = [I, I, S, I, I, PP, PP, QP, QP, PP, PP, ctypes.c_uint, P, I, P]
+        L.fc_p2p_allreduce.restype = I
+        L.fc_p2p_allreduce_emulated.restype = I
         L.fc_host_device_pointer.argtypes = [P, ctypes.POINTER(P)]
         L.fc_host_device_pointer.restype = I
         L.fc_ipc_export.argtypes = [P, ctypes.c_char_p, ctypes.POINTER(S)]
@@ -193,6 +198,10 @@ class PeerQBuf(QBuf):
     def struct(self):
         return fc_qbuf(self.codes, self.scales, self.zps)
 
+    def bytes(self) -> int:
+        cb, nb = fc_payload_sizes(self.n, self.bits, self.block)
+        return cb + 5 * nb
+
 
 FC_IPC_HANDLE_BYTES = 64
 
@@ -216,6 +225,44 @@ def fc_ipc_open(handle: bytes) -> int:
 
 def fc_ipc_close(base: int) -> None:
     _check(_lib().fc_ipc_close(ctypes.c_void_p(base)), "fc_ipc_close")
+
+
+def _addr(v) -> int:
+    """Device address of a tensor or of a raw address."""
+    return v if isinstance(v, int) else _dev_ptr(v, "pointer")
+
+
+def _p2p_tables(P, s1, s2, ctr1, ctr2):
+    if len(s1) != P * P or len(s2) != P or len(ctr1) != P or len(ctr2) != P:
+        raise ValueError("s1 holds P*P payloads (s1[p*P + c]); s2, ctr1, ctr2 hold P entries")
+    return ((fc_qbuf * (P * P))(*[q.struct() for q in s1]), (fc_qbuf * P)(*[q.struct() for q in s2]),
+            (ctypes.c_void_p * P)(*[_addr(c) for c in ctr1]), (ctypes.c_void_p * P)(*[_addr(c) for c in ctr2]))
+
+
+def fc_p2p_allreduce(rank: int, x, y, bits: int, block: int, s1, s2, ctr1, ctr2, epoch: int, status,
+                     ctas_per_rank: int = 0, stream=None):
+    """One rank's one-kernel P-GPU all-reduce (see include/fc.h): s1 = P*P payloads (rank p's
+    chunk c at p*P + c), s2 = P owners' payloads, ctr1/ctr2 = P counters (tensors or addresses)."""
+    P = len(s2)
+    a1, a2, c1, c2 = _p2p_tables(P, s1, s2, ctr1, ctr2)
+    _check(_lib().fc_p2p_allreduce(rank, P, _dtype_code(x), x.numel(), bits, block,
+                                   ctypes.c_void_p(_dev_ptr(x, "x")), ctypes.c_void_p(_dev_ptr(y, "y")),
+                                   a1, a2, c1, c2, epoch, ctypes.c_void_p(_addr(status)), ctas_per_rank,
+                                   _stream(stream)), "fc_p2p_allreduce")
+    return y
+
+
+def fc_p2p_allreduce_emulated(xs, ys, bits: int, block: int, s1, s2, ctr1, ctr2, epoch: int, status,
+                              ctas_per_rank: int = 0, stream=None):
+    """All P ranks of fc_p2p_allreduce in one cooperative launch on the current GPU."""
+    P = len(xs)
+    a1, a2, c1, c2 = _p2p_tables(P, s1, s2, ctr1, ctr2)
+    xp = (ctypes.c_void_p * P)(*[_dev_ptr(x, "x") for x in xs])
+    yp = (ctypes.c_void_p * P)(*[_dev_ptr(y, "y") for y in ys])
+    _check(_lib().fc_p2p_allreduce_emulated(P, _dtype_code(xs[0]), xs[0].numel(), bits, block, xp, yp, a1, a2,
+                                            c1, c2, epoch, ctypes.c_void_p(_addr(status)), ctas_per_rank,
+                                            _stream(stream)), "fc_p2p_allreduce_emulated")
+    return ys
 
 
 def fc_quantize(x, bits: int, block: int, out: QBuf | None = None, stream=None) -> QBuf:

@@ -15,6 +15,7 @@
 #include "../../include/fc.h"
 #include "fc_gemm.cuh"
 #include "fc_kernels.cuh"
+#include "fc_p2p_args.cuh"
 
 namespace {
 
@@ -466,6 +467,105 @@ const GemmFnT kGemmPair[2][2][3] = {
 
 }  // namespace
 
+// ---- the one-kernel P-GPU all-reduce -------------------------------------------
+namespace {
+using P2PLaunch = cudaError_t (*)(const fc::P2PArgs&, int, cudaStream_t);
+using P2PCtas = cudaError_t (*)(int*);
+#define FC_P2P_ROW(T, B, EMU)                                                                   \
+    {fc::launch_p2p<T, B, 2, EMU>, fc::launch_p2p<T, B, 4, EMU>, fc::launch_p2p<T, B, 8, EMU>}
+#define FC_P2P_CTAS(T, B, EMU)                                                                  \
+    {fc::p2p_max_ctas<T, B, 2, EMU>, fc::p2p_max_ctas<T, B, 4, EMU>, fc::p2p_max_ctas<T, B, 8, EMU>}
+// [emulated][dtype][bits == 4][P = 2, 4, 8]
+const P2PLaunch kP2P[2][2][2][3] = {
+    {{FC_P2P_ROW(__half, 8, false), FC_P2P_ROW(__half, 4, false)},
+     {FC_P2P_ROW(__nv_bfloat16, 8, false), FC_P2P_ROW(__nv_bfloat16, 4, false)}},
+    {{FC_P2P_ROW(__half, 8, true), FC_P2P_ROW(__half, 4, true)},
+     {FC_P2P_ROW(__nv_bfloat16, 8, true), FC_P2P_ROW(__nv_bfloat16, 4, true)}},
+};
+const P2PCtas kP2PCtas[2][2][2][3] = {
+    {{FC_P2P_CTAS(__half, 8, false), FC_P2P_CTAS(__half, 4, false)},
+     {FC_P2P_CTAS(__nv_bfloat16, 8, false), FC_P2P_CTAS(__nv_bfloat16, 4, false)}},
+    {{FC_P2P_CTAS(__half, 8, true), FC_P2P_CTAS(__half, 4, true)},
+     {FC_P2P_CTAS(__nv_bfloat16, 8, true), FC_P2P_CTAS(__nv_bfloat16, 4, true)}},
+};
+#undef FC_P2P_CTAS
+#undef FC_P2P_ROW
+
+fc_status p2p_common(bool emu, int rank, int P, fc_dtype dtype, size_t n, int bits, int block,
+                     const void* const* x, void* const* y, const fc_qbuf* s1, const fc_qbuf* s2,
+                     unsigned int* const* ctr1, unsigned int* const* ctr2, unsigned int epoch, int* status,
+                     int ctas_per_rank, void* stream)
+{
+    const int pi = P == 2 ? 0 : P == 4 ? 1 : P == 8 ? 2 : -1;
+    if (pi < 0 || !valid_bits(bits) || !valid_block(block) || (dtype != FC_FP16 && dtype != FC_BF16) ||
+        n % ((size_t)P * (size_t)block) != 0 || (!emu && (rank < 0 || rank >= P)) || epoch == 0 ||
+        ctas_per_rank < 0)
+        return FC_ERR_INVALID_ARG;
+    if (n == 0)
+        return FC_OK;
+    if (x == nullptr || y == nullptr || s1 == nullptr || s2 == nullptr || ctr1 == nullptr || ctr2 == nullptr ||
+        status == nullptr)
+        return FC_ERR_INVALID_ARG;
+    const size_t m = n / (size_t)P;
+    fc::P2PArgs a{};
+    const int nio = emu ? P : 1;
+    for (int i = 0; i < nio; i++) {
+        if (x[i] == nullptr || y[i] == nullptr)
+            return FC_ERR_INVALID_ARG;
+        if (!aligned16(x[i]) || !aligned16(y[i]))
+            return FC_ERR_MISALIGNED;
+        a.x[i] = x[i];
+        a.y[i] = y[i];
+    }
+    Range scratch[3];
+    for (int p = 0; p < P; p++) {
+        for (int c = 0; c < P; c++) {
+            fc_status st = check_qbuf(&s1[p * P + c], m, bits, block, scratch);
+            if (st != FC_OK)
+                return st;
+            a.s1[p][c] = qptr(&s1[p * P + c]);
+        }
+        fc_status st = check_qbuf(&s2[p], m, bits, block, scratch);
+        if (st != FC_OK)
+            return st;
+        a.s2[p] = qptr(&s2[p]);
+        if (ctr1[p] == nullptr || ctr2[p] == nullptr)
+            return FC_ERR_INVALID_ARG;
+        if ((reinterpret_cast<uintptr_t>(ctr1[p]) & 3u) || (reinterpret_cast<uintptr_t>(ctr2[p]) & 3u))
+            return FC_ERR_MISALIGNED;
+        a.ctr1[p] = ctr1[p];
+        a.ctr2[p] = ctr2[p];
+    }
+    if (reinterpret_cast<uintptr_t>(status) & 3u)
+        return FC_ERR_MISALIGNED;
+    a.status = status;
+    a.m = m;
+    a.block = block;
+    a.rank = emu ? 0 : rank;
+    a.epoch = epoch;
+    // co-resident CTAs: all ranks' CTAs wait on each other
+    int max_ctas = 0;
+    cudaError_t e = kP2PCtas[emu][dtype][bits == 4][pi](&max_ctas);
+    if (e != cudaSuccess)
+        return cuda_fail(e);
+    const int ranks_here = emu ? P : 1;
+    const size_t tiles = (n + (size_t)fc::P2P_TILE - 1) / (size_t)fc::P2P_TILE;
+    int cpr = max_ctas / ranks_here;
+    if (ctas_per_rank > 0 && ctas_per_rank < cpr)
+        cpr = ctas_per_rank;
+    if ((size_t)cpr > tiles)
+        cpr = (int)tiles;
+    if (cpr < 1)
+        return FC_ERR_UNSUPPORTED;
+    a.cpr = cpr;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    e = cudaMemsetAsync(status, 0, sizeof(int), st);
+    if (e == cudaSuccess)
+        e = kP2P[emu][dtype][bits == 4][pi](a, cpr * ranks_here, st);
+    return e == cudaSuccess ? FC_OK : cuda_fail(e);
+}
+}  // namespace
+
 extern "C" {
 
 fc_status fc_gemm_quantize(const void* a, const void* w, fc_dtype dtype, int M, int N, int K, int bits, int block,
@@ -531,6 +631,26 @@ fc_status fc_host_device_pointer(const void* host, void** device)
     }
     *device = d;
     return FC_OK;
+}
+
+
+// ---- the one-kernel P-GPU all-reduce (entry points) ---------------------------
+fc_status fc_p2p_allreduce(int rank, int P, fc_dtype dtype, size_t n, int bits, int block, const void* x, void* y,
+                           const fc_qbuf* s1, const fc_qbuf* s2, unsigned int* const* ctr1,
+                           unsigned int* const* ctr2, unsigned int epoch, int* status, int ctas_per_rank,
+                           void* stream)
+{
+    return p2p_common(false, rank, P, dtype, n, bits, block, &x, &y, s1, s2, ctr1, ctr2, epoch, status,
+                      ctas_per_rank, stream);
+}
+
+fc_status fc_p2p_allreduce_emulated(int P, fc_dtype dtype, size_t n, int bits, int block, const void* const* x,
+                                    void* const* y, const fc_qbuf* s1, const fc_qbuf* s2,
+                                    unsigned int* const* ctr1, unsigned int* const* ctr2, unsigned int epoch,
+                                    int* status, int ctas_per_rank, void* stream)
+{
+    return p2p_common(true, 0, P, dtype, n, bits, block, x, y, s1, s2, ctr1, ctr2, epoch, status, ctas_per_rank,
+                      stream);
 }
 
 // ---- peer memory (CUDA IPC) for the P-GPU deployment -------------------------

@@ -213,6 +213,49 @@ fc_status fc_ipc_open(const void* handle, void** base);
  * completed).  Errors: FC_ERR_INVALID_ARG for NULL; FC_ERR_CUDA. */
 fc_status fc_ipc_close(void* base);
 
+/* The P-GPU all-reduce as ONE kernel per rank (page: TL;DR, the fused
+ * quantize -> reduce-scatter -> all-gather all-reduce; Fig. 3, one partial per
+ * tensor-parallel rank).  Rank r's kernel quantizes its partial x (n elements)
+ * chunk by chunk into its step-1 payloads, counts on its phase-1 counter, waits
+ * for every rank's count, reduce-scatters chunk r by reading every rank's
+ * step-1 payload of chunk r (peer memory), writes its step-2 payload, counts on
+ * its phase-2 counter, waits, and all-gathers every owner's step-2 payload into
+ * y -- bit-identical to fc_quantized_allreduce on the P partials.
+ *   rank, P     this rank, P in {2, 4, 8};
+ *   x, y        this rank's input and output (device, n fp16/bf16 values);
+ *   s1          host array of P*P payloads: s1[p*P + c] = rank p's step-1
+ *               payload of chunk c (m = n/P elements each), as this process
+ *               addresses it (own memory, or a peer mapping from fc_ipc_open);
+ *   s2          host array of P payloads: s2[c] = owner c's step-2 payload of
+ *               chunk c (m elements);
+ *   ctr1, ctr2  host arrays of P device pointers to rank p's phase counters
+ *               (uint32, zero before the first call, never reset);
+ *   epoch       1 on the first call with fresh counters, then 2, 3, ...: the
+ *               k-th call waits for k * (CTAs per rank) counts;
+ *   status      device int of this rank: set to 0 on the stream, OR-ed with 1
+ *               when a wait gave up after 2 s (a missing or failed peer); the
+ *               outputs are then invalid and the counters no longer agree;
+ *   ctas_per_rank  0 = as many as can be co-resident (the usual), else a cap;
+ *               every rank must use the same value.
+ * The kernel is launched cooperatively (its CTAs wait on each other and on the
+ * peers'): no other kernel that waits on this rank may share the GPU.  Requires
+ * n % (P*block) == 0, 16-byte-aligned payloads, 4-byte-aligned counters.  The
+ * ranks' calls must use the same n, bits, block, dtype and epoch. */
+fc_status fc_p2p_allreduce(int rank, int P, fc_dtype dtype, size_t n, int bits, int block, const void* x, void* y,
+                           const fc_qbuf* s1, const fc_qbuf* s2, unsigned int* const* ctr1,
+                           unsigned int* const* ctr2, unsigned int epoch, int* status, int ctas_per_rank,
+                           void* stream);
+
+/* fc_p2p_allreduce for all P ranks at once on the current GPU: one
+ * cooperative launch whose CTAs play every rank (the protocol of the P-GPU
+ * kernel, run where one GPU holds every rank's buffers).  x and y are host
+ * arrays of P device pointers (rank p's input and output); s1, s2, ctr1, ctr2
+ * and status as above (one status word for all ranks). */
+fc_status fc_p2p_allreduce_emulated(int P, fc_dtype dtype, size_t n, int bits, int block, const void* const* x,
+                                    void* const* y, const fc_qbuf* s1, const fc_qbuf* s2,
+                                    unsigned int* const* ctr1, unsigned int* const* ctr2, unsigned int epoch,
+                                    int* status, int ctas_per_rank, void* stream);
+
 /* Static description of a status code. */
 const char* fc_status_string(fc_status status);
 

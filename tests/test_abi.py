@@ -122,3 +122,23 @@ def test_ipc_validation():
     assert lib.fc_host_device_pointer(ctypes.c_void_p(A), None) == fc.FC_ERR_INVALID_ARG
     with pytest.raises(ValueError):
         fc.fc_ipc_open(b"short")
+
+
+def test_p2p_validation():
+    lib = fc.library()
+    P = 2
+    s1 = (fc.fc_qbuf * 4)(*[qb(A + i * 0x1000000) for i in range(4)])
+    s2 = (fc.fc_qbuf * 2)(*[qb(A + (4 + i) * 0x1000000) for i in range(2)])
+    ctr = (ctypes.c_void_p * 2)(A + 0x70000000, A + 0x70000010)
+    st = ctypes.c_void_p(A + 0x70000100)
+    x, y = ctypes.c_void_p(A + 0x60000000), ctypes.c_void_p(A + 0x68000000)
+    call = lambda **kw: lib.fc_p2p_allreduce(kw.get("rank", 0), kw.get("P", P), 0, kw.get("n", 4096), kw.get("bits", 8),
+                                             128, x, y, s1, s2, ctr, ctr, kw.get("epoch", 1), st, 0, None)
+    assert call(P=3) == fc.FC_ERR_INVALID_ARG          # P in {2, 4, 8}
+    assert call(rank=2) == fc.FC_ERR_INVALID_ARG
+    assert call(bits=5) == fc.FC_ERR_INVALID_ARG
+    assert call(n=4096 + 128) == fc.FC_ERR_INVALID_ARG  # n % (P*block)
+    assert call(epoch=0) == fc.FC_ERR_INVALID_ARG
+    assert call(n=0) == fc.FC_OK
+    assert lib.fc_p2p_allreduce(0, 2, 0, 4096, 8, 128, x, y, None, s2, ctr, ctr, 1, st, 0, None) == fc.FC_ERR_INVALID_ARG
+    assert lib.fc_p2p_allreduce(0, 2, 0, 4096, 8, 128, x, y, s1, s2, ctr, ctr, 1, None, 0, None) == fc.FC_ERR_INVALID_ARG
