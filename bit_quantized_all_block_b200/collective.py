@@ -28,13 +28,20 @@ bit-identical to `fc_quantized_allreduce` on the P partials.
 
 The device operations come from an `ops` object (`CudaOps`: the library's
 kernels, buffers in GPU memory, peers mapped with fc_ipc_open).
+
+With one_kernel=True (one GPU per rank) each call is instead a single launch
+of fc_p2p_allreduce: the same three steps inside one cooperative kernel per
+rank, the ranks synchronised by counters in their arenas (system-scope
+atomics and acquire loads through the peer mappings, bounded waits) instead
+of host barriers.  Kernels of different ranks then wait on each other, so
+this mode refuses ranks that share a GPU.
 """
 from __future__ import annotations
 
 from dataclasses import dataclass
 
-from . import (PeerQBuf, fc_ag_dequant, fc_ipc_close, fc_ipc_export, fc_ipc_open, fc_payload_sizes,
-               fc_quantize, fc_rs_dequant_sum_requant)
+from . import (PeerQBuf, fc_ag_dequant, fc_ipc_close, fc_ipc_export, fc_ipc_open, fc_p2p_allreduce,
+               fc_payload_sizes, fc_quantize, fc_rs_dequant_sum_requant)
 
 ALIGN = 256
 
@@ -72,6 +79,7 @@ class Layout:
 
         self._step1 = [(take(cb), take(4 * nb), take(nb)) for _ in range(P)]
         self._step2 = (take(cb), take(4 * nb), take(nb))
+        self.counters = take(8)          # phase-1 and phase-2 counters of the one-kernel mode (uint32 each)
         self.nbytes = off
 
     def step1(self, holder: int, c: int) -> PayloadRef:
@@ -81,6 +89,12 @@ class Layout:
     def step2(self, owner: int) -> PayloadRef:
         """The step-2 payload of chunk `owner`, held by its owner."""
         return PayloadRef(owner, *self._step2, self.m)
+
+
+def ranks_share_a_device(device_ids) -> bool:
+    """Whether two ranks report the same GPU (their one-kernel calls would wait
+    on each other on one device, which nothing guarantees to make progress)."""
+    return len(set(device_ids)) != len(device_ids)
 
 
 def schedule(rank: int, layout: Layout):
@@ -107,7 +121,11 @@ class CudaOps:
         self.opened = []
 
     def alloc(self, nbytes: int):
-        self.arena = self.torch.empty(max(nbytes, ALIGN), dtype=self.torch.uint8, device=self.device)
+        # zeroed: the one-kernel mode's counters start at 0
+        self.arena = self.torch.zeros(max(nbytes, ALIGN), dtype=self.torch.uint8, device=self.device)
+
+    def device_id(self) -> str:
+        return str(self.torch.cuda.get_device_properties(self.device).uuid)
 
     def export(self):
         return fc_ipc_export(self.arena.data_ptr())
@@ -156,7 +174,7 @@ class QuantizedAllReduce:
     partial x (n elements, flat) writes the all-reduced result to y (default: a
     new tensor) and returns it; every rank receives the same bits."""
 
-    def __init__(self, n: int, bits: int, block: int, group=None, ops=None):
+    def __init__(self, n: int, bits: int, block: int, group=None, ops=None, one_kernel: bool = False):
         import torch.distributed as dist
         self.dist = dist
         self.group = group if group is not None else dist.group.WORLD
@@ -174,9 +192,17 @@ class QuantizedAllReduce:
         self.ops.alloc(self.layout.nbytes)
         exported = [None] * self.P
         dist.all_gather_object(exported, self.ops.export(), group=self.host)
+        self.one_kernel = one_kernel
+        if one_kernel:
+            ids = [None] * self.P
+            dist.all_gather_object(ids, self.ops.device_id(), group=self.host)
+            if ranks_share_a_device(ids):
+                raise ValueError("one_kernel needs one GPU per rank: the ranks' kernels wait on each other")
+            self.epoch = 0
+            self.status = self.ops.torch.zeros(1, dtype=self.ops.torch.int32, device=self.ops.device)
         self.ops.attach(self.rank, exported)
         self.plan = schedule(self.rank, self.layout)
-        self.barrier()      # every mapping is in place before the first read
+        self.barrier()      # every mapping is in place (and every counter zero) before the first read
 
     def barrier(self):
         self.ops.sync()
@@ -189,6 +215,8 @@ class QuantizedAllReduce:
             raise ValueError(f"expected {L.n} elements, got {x.shape[0]}")
         if y is None:
             y = self.ops.new_output(x)
+        if self.one_kernel:
+            return self._one_kernel_call(x, y)
         quantize, (ins, out), ag = self.plan
         for c, ref in enumerate(quantize):
             self.ops.quantize(x, c * L.m, L.m, ref, b, B)
@@ -198,6 +226,20 @@ class QuantizedAllReduce:
         for c, ref in enumerate(ag):
             self.ops.ag(ref, y, c * L.m, L.m, b, B)
         return y
+
+    def _one_kernel_call(self, x, y):
+        L, P = self.layout, self.P
+        self.epoch += 1
+        s1 = [self.ops.qbuf(L.step1(p, c), self.bits, self.block) for p in range(P) for c in range(P)]
+        s2 = [self.ops.qbuf(L.step2(c), self.bits, self.block) for c in range(P)]
+        ctr1 = [self.ops.base[p] + L.counters for p in range(P)]
+        ctr2 = [self.ops.base[p] + L.counters + 4 for p in range(P)]
+        fc_p2p_allreduce(self.rank, x, y, self.bits, self.block, s1, s2, ctr1, ctr2, self.epoch, self.status)
+        return y
+
+    def last_status(self) -> int:
+        """One-kernel mode: 0, or 1 if a wait of the last call gave up (synchronizes)."""
+        return int(self.status.item()) if self.one_kernel else 0
 
     def close(self):
         """Unmap the peers' arenas (collective: every rank, after its last call)."""

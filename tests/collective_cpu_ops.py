@@ -21,6 +21,9 @@ class OracleOps:
     def export(self):
         return self.shm.name
 
+    def device_id(self) -> str:
+        return "cpu"
+
     def attach(self, rank: int, exported: list):
         for r, name in enumerate(exported):
             self.peers[r] = self.shm if r == rank else shared_memory.SharedMemory(name=name)

@@ -84,3 +84,17 @@ def test_ranks_reproduce_the_one_process_allreduce(world, bits, block, dtype):
         y_ref, _, _ = oracle.allreduce(list(xs), dtype, bits, block)
         for r in range(world):
             assert np.array_equal(out[r][k], y_ref), f"rank {r}, call {k}"
+
+
+def test_one_kernel_mode_refuses_ranks_on_one_device():
+    from bit_quantized_all_block_b200.collective import ranks_share_a_device
+    assert ranks_share_a_device(["GPU-a", "GPU-a"])
+    assert ranks_share_a_device(["GPU-a", "GPU-b", "GPU-a", "GPU-c"])
+    assert not ranks_share_a_device(["GPU-a", "GPU-b", "GPU-c", "GPU-d"])
+
+
+def test_layout_reserves_aligned_counters():
+    L = Layout(8192, 4, 8, 128)
+    assert L.counters % ALIGN == 0 and L.counters + 8 <= L.nbytes
+    last = L.step2(0)
+    assert L.counters >= last.zps + 2048 // 128

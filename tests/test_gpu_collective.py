@@ -69,3 +69,27 @@ def test_ranks_match_the_oracle(world, bits, block, dtype, rows):
             got = out[r][k]
             bad = np.nonzero(got != y_ref)[0]
             assert bad.size == 0, f"rank {r}, call {k}: {bad.size} outputs differ, first at {bad[:8]}"
+
+
+def _rank_one_kernel(rank, world, port, out):
+    from bit_quantized_all_block_b200.collective import QuantizedAllReduce
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    torch.cuda.set_device(0)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        try:
+            QuantizedAllReduce(2 * 128 * 4, 8, 128, one_kernel=True)
+            out[rank] = "built"
+        except ValueError:
+            out[rank] = "refused"
+    finally:
+        dist.destroy_process_group()
+
+
+def test_one_kernel_mode_refuses_ranks_that_share_a_gpu():
+    """The one-kernel mode's kernels wait on each other; on a shared GPU that
+    could never be guaranteed to progress, so construction is refused (before
+    any launch)."""
+    out = mp.get_context("spawn").Manager().dict()
+    mp.start_processes(_rank_one_kernel, args=(2, _free_port(), out), nprocs=2, join=True, start_method="spawn")
+    assert out[0] == "refused" and out[1] == "refused"
