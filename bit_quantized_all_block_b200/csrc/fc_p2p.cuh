@@ -22,7 +22,8 @@
 // Visibility: a CTA's payload writes are ordered before its count by a CTA
 // barrier and a system-scope fence in the counting thread; a waiting thread
 // reads counters with system-scope acquire loads, then releases its CTA with
-// a barrier.  Every wait gives up after 2 s of %globaltimer, ORs 1 into the
+// a barrier; payloads written during the launch are then read with coherent
+// L2 loads (never through the read-only path).  Every wait gives up after 2 s of %globaltimer, ORs 1 into the
 // status word and skips the rest of the call, so a missing peer ends the call
 // with an error instead of a hang.
 //
@@ -87,6 +88,30 @@ __device__ __forceinline__ bool p2p_wait(unsigned int* const* ctrs, unsigned int
     }
     __syncthreads();
     return *abort_smem == 0;
+}
+
+// A thread's E codes of a payload written during this launch (by other CTAs
+// or other GPUs): coherent loads that bypass L1 and the read-only path, which
+// assume data that does not change while the kernel runs.
+template <int BITS, int NC>
+__device__ __forceinline__ void load_codes_cg(const uint8_t* codes, size_t e, uint32_t* w)
+{
+    constexpr int NW = NC * BITS / 4;
+    const uint8_t* p = codes + e * BITS / 8;
+    if constexpr (NW % 4 == 0) {
+#pragma unroll
+        for (int i = 0; i < NW; i += 4) {
+            const uint4 v = __ldcg(reinterpret_cast<const uint4*>(p + 4 * i));
+            w[i] = v.x;
+            w[i + 1] = v.y;
+            w[i + 2] = v.z;
+            w[i + 3] = v.w;
+        }
+    } else {
+        const uint2 v = __ldcg(reinterpret_cast<const uint2*>(p));
+        w[0] = v.x;
+        w[1] = v.y;
+    }
 }
 
 template <class T, int BITS, int P, bool EMU>
@@ -163,9 +188,9 @@ __global__ void __launch_bounds__(P2P_THREADS) k_p2p(const __grid_constant__ P2P
             float s = 1.0f, mz = FC_MAGIC;
             if (valid) {
                 const QPtr& q = a.s1[r][rank];
-                load_thread_codes<BITS, NC>(q.codes, el, w);
-                s = q.scales[k];
-                mz = __uint_as_float(FC_MAGIC_BITS + q.zps[k]);
+                load_codes_cg<BITS, NC>(q.codes, el, w);
+                s = __ldcg(q.scales + k);
+                mz = __uint_as_float(FC_MAGIC_BITS + __ldcg(q.zps + k));
             } else {
 #pragma unroll
                 for (int i = 0; i < NW; i++)
@@ -211,9 +236,9 @@ __global__ void __launch_bounds__(P2P_THREADS) k_p2p(const __grid_constant__ P2P
         const QPtr& q = a.s2[ch];
         const size_t k = el >> lg_block;
         uint32_t w[NW];
-        load_thread_codes<BITS, NC>(q.codes, el, w);
-        const float s = q.scales[k];
-        const float mz = __uint_as_float(FC_MAGIC_BITS + q.zps[k]);
+        load_codes_cg<BITS, NC>(q.codes, el, w);
+        const float s = __ldcg(q.scales + k);
+        const float mz = __uint_as_float(FC_MAGIC_BITS + __ldcg(q.zps + k));
         uint4 ov[NC];
 #pragma unroll
         for (int c = 0; c < NC; c++) {
