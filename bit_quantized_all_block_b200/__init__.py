@@ -29,6 +29,10 @@ FC_ERR_INVALID_ARG = 1
 FC_ERR_UNSUPPORTED = 2
 FC_ERR_MISALIGNED = 3
 FC_ERR_CUDA = 4
+FC_ERR_TOO_LARGE = 5
+
+# bytes of static device scratch behind fc_p2p_allreduce_emulated_noalloc
+FC_NOALLOC_SCRATCH_BYTES = 16 << 20
 
 FC_FP16 = 0
 FC_BF16 = 1
@@ -76,6 +80,8 @@ def _lib():
         L.fc_p2p_allreduce_emulated.argtypes = [I, I, S, I, I, PP, PP, QP, QP, PP, PP, ctypes.c_uint, P, I, P]
         L.fc_p2p_allreduce.restype = I
         L.fc_p2p_allreduce_emulated.restype = I
+        L.fc_p2p_allreduce_emulated_noalloc.argtypes = [I, I, S, I, I, PP, PP, P, P]
+        L.fc_p2p_allreduce_emulated_noalloc.restype = I
         L.fc_host_device_pointer.argtypes = [P, ctypes.POINTER(P)]
         L.fc_host_device_pointer.restype = I
         L.fc_ipc_export.argtypes = [P, ctypes.c_char_p, ctypes.POINTER(S)]
@@ -262,6 +268,21 @@ def fc_p2p_allreduce_emulated(xs, ys, bits: int, block: int, s1, s2, ctr1, ctr2,
     _check(_lib().fc_p2p_allreduce_emulated(P, _dtype_code(xs[0]), xs[0].numel(), bits, block, xp, yp, a1, a2,
                                             c1, c2, epoch, ctypes.c_void_p(_addr(status)), ctas_per_rank,
                                             _stream(stream)), "fc_p2p_allreduce_emulated")
+    return ys
+
+
+def fc_p2p_allreduce_emulated_noalloc(xs, ys, bits: int, block: int, status=None, stream=None):
+    """fc_p2p_allreduce_emulated with its payloads and counters in the library's static
+    device scratch, for callers that must not allocate device memory (include/fc.h).
+    ``ys`` are the P caller-owned outputs; ``status`` an optional device int (tensor or address)."""
+    P = len(xs)
+    if len(ys) != P:
+        raise ValueError("xs and ys hold one tensor per rank")
+    xp = (ctypes.c_void_p * P)(*[_dev_ptr(x, "x") for x in xs])
+    yp = (ctypes.c_void_p * P)(*[_dev_ptr(y, "y") for y in ys])
+    st = ctypes.c_void_p(_addr(status)) if status is not None else None
+    _check(_lib().fc_p2p_allreduce_emulated_noalloc(P, _dtype_code(xs[0]), xs[0].numel(), bits, block, xp, yp, st,
+                                                    _stream(stream)), "fc_p2p_allreduce_emulated_noalloc")
     return ys
 
 

@@ -710,6 +710,7 @@ const char* fc_status_string(fc_status status)
     case FC_ERR_UNSUPPORTED: return "unsupported combination";
     case FC_ERR_MISALIGNED: return "device pointer not 16-byte aligned";
     case FC_ERR_CUDA: return "CUDA error (see fc_last_cuda_error)";
+    case FC_ERR_TOO_LARGE: return "problem needs more than the library's fixed scratch memory";
     }
     return "unknown status";
 }
@@ -717,3 +718,95 @@ const char* fc_status_string(fc_status status)
 int fc_last_cuda_error(void) { return g_last_cuda_error; }
 
 }  // extern "C"
+
+// ---- the all-reduce for callers that cannot allocate device memory ------------
+// fc_p2p_allreduce_emulated with its scratch (step-1 and step-2 payloads, phase
+// counters, status word) in a fixed array of static device memory instead of
+// caller buffers.  Layout, every piece 256-byte aligned:
+//   [0, 256)  ctr1[0..P) at words 0..7, ctr2[0..P) at words 8..15, status at 16
+//   then s1[p][c] for p, c in [0, P) and s2[c] for c in [0, P), each
+//   codes R(m*bits/8), scales R(4*m/block), zps R(m/block).
+namespace {
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[FC_NOALLOC_SCRATCH_BYTES];
+
+constexpr size_t kNoallocHeader = 256;
+constexpr int kNoallocMaxDevices = 64;
+std::mutex g_noalloc_mu;
+unsigned char* g_noalloc_addr[kNoallocMaxDevices];   // device address of the array, per device
+
+size_t round256(size_t v) { return (v + 255) & ~(size_t)255; }
+
+// Device address of the scratch array on the current device (looked up once per device).
+fc_status noalloc_scratch(unsigned char** out)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return cuda_fail(e);
+    if (dev < 0 || dev >= kNoallocMaxDevices)
+        return FC_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (g_noalloc_addr[dev] == nullptr) {
+        void* ptr = nullptr;
+        e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+        if (e != cudaSuccess)
+            return cuda_fail(e);
+        g_noalloc_addr[dev] = static_cast<unsigned char*>(ptr);
+    }
+    *out = g_noalloc_addr[dev];
+    return FC_OK;
+}
+
+}  // namespace
+
+extern "C" fc_status fc_p2p_allreduce_emulated_noalloc(int P, fc_dtype dtype, size_t n, int bits, int block,
+                                                       const void* const* x, void* const* y, int* status,
+                                                       void* stream)
+{
+    if ((P != 2 && P != 4 && P != 8) || !valid_bits(bits) || !valid_block(block) ||
+        (dtype != FC_FP16 && dtype != FC_BF16) || n % ((size_t)P * (size_t)block) != 0)
+        return FC_ERR_INVALID_ARG;
+    if (n == 0)
+        return FC_OK;
+    if (x == nullptr || y == nullptr)
+        return FC_ERR_INVALID_ARG;
+    // the step-1 codes alone take n*bits/8 >= n/2 bytes: this bound keeps the sums below exact
+    if (n / 2 > (size_t)FC_NOALLOC_SCRATCH_BYTES)
+        return FC_ERR_TOO_LARGE;
+    const size_t m = n / (size_t)P;
+    const size_t codes = round256(m * (size_t)bits / 8), scales = round256(4 * (m / (size_t)block)),
+                 zps = round256(m / (size_t)block);
+    const size_t piece = codes + scales + zps;
+    if (kNoallocHeader + (size_t)P * (size_t)(P + 1) * piece > (size_t)FC_NOALLOC_SCRATCH_BYTES)
+        return FC_ERR_TOO_LARGE;
+    unsigned char* base = nullptr;
+    fc_status st = noalloc_scratch(&base);
+    if (st != FC_OK)
+        return st;
+    fc_qbuf s1[fc::FC_MAX_P * fc::FC_MAX_P], s2[fc::FC_MAX_P];
+    unsigned int* ctr1[fc::FC_MAX_P];
+    unsigned int* ctr2[fc::FC_MAX_P];
+    unsigned int* words = reinterpret_cast<unsigned int*>(base);
+    unsigned char* cur = base + kNoallocHeader;
+    auto carve = [&](fc_qbuf* q) {
+        q->codes = cur;
+        q->scales = reinterpret_cast<float*>(cur + codes);
+        q->zps = cur + codes + scales;
+        cur += piece;
+    };
+    for (int i = 0; i < P * P; i++)
+        carve(&s1[i]);
+    for (int c = 0; c < P; c++) {
+        carve(&s2[c]);
+        ctr1[c] = words + c;
+        ctr2[c] = words + 8 + c;
+    }
+    int* own_status = reinterpret_cast<int*>(words + 16);
+    // counters and the status word start at zero on every call (epoch 1)
+    cudaError_t e = cudaMemsetAsync(base, 0, kNoallocHeader, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess)
+        return cuda_fail(e);
+    return p2p_common(true, 0, P, dtype, n, bits, block, x, y, s1, s2, ctr1, ctr2, 1u,
+                      status != nullptr ? status : own_status, 0, stream);
+}

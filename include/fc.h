@@ -77,7 +77,8 @@ typedef enum {
     FC_ERR_INVALID_ARG = 1, /* bad size, bits, block, P, NULL or overlapping buffers */
     FC_ERR_UNSUPPORTED = 2, /* a combination this build does not provide          */
     FC_ERR_MISALIGNED = 3,  /* a device pointer is not 16-byte aligned             */
-    FC_ERR_CUDA = 4         /* a CUDA call failed; see fc_last_cuda_error()       */
+    FC_ERR_CUDA = 4,        /* a CUDA call failed; see fc_last_cuda_error()       */
+    FC_ERR_TOO_LARGE = 5    /* needs more than the library's fixed scratch memory */
 } fc_status;
 
 typedef enum { FC_FP16 = 0, FC_BF16 = 1 } fc_dtype;
@@ -255,6 +256,50 @@ fc_status fc_p2p_allreduce_emulated(int P, fc_dtype dtype, size_t n, int bits, i
                                     void* const* y, const fc_qbuf* s1, const fc_qbuf* s2,
                                     unsigned int* const* ctr1, unsigned int* const* ctr2, unsigned int epoch,
                                     int* status, int ctas_per_rank, void* stream);
+
+/* fc_p2p_allreduce_emulated for callers that cannot allocate device memory.
+ * The page has no counterpart: this is a convenience of this library.
+ *
+ * Who needs it: code that must not call cudaMalloc/cudaFree at the point
+ * where it runs the all-reduce -- a plugin whose host framework owns all
+ * device memory and forbids allocation inside its execute callback, a serving
+ * loop that cannot afford the device-wide synchronisation cudaFree implies,
+ * or a process whose memory a caching allocator has already reserved.  Such
+ * a caller holds its inputs and outputs but has nowhere to put the wire
+ * payloads and the phase counters the all-reduce works through.
+ *
+ * This entry point keeps all of that scratch (every rank's step-1 chunk
+ * payloads, every owner's step-2 payload, the 2*P phase counters and a
+ * status word) in one array of FC_NOALLOC_SCRATCH_BYTES bytes of static
+ * device memory inside the library.  Every GPU on which the library's module
+ * is loaded holds that array until the process exits.  The call allocates
+ * nothing: it clears the counters and the status word with cudaMemsetAsync
+ * on `stream` and runs the same cooperative kernel as
+ * fc_p2p_allreduce_emulated (epoch 1 on the cleared counters), so y equals
+ * what fc_p2p_allreduce_emulated and fc_quantized_allreduce produce, bit for
+ * bit.
+ *   P, dtype, n, bits, block, x, y   as for fc_p2p_allreduce_emulated
+ *                                    (P in {2, 4, 8}; x and y host arrays of
+ *                                    P device pointers; n per rank);
+ *   status   device int, or NULL: set to 0 on the stream, OR-ed with 1 if a
+ *            wait inside the kernel gave up (outputs then invalid).  With
+ *            NULL that flag stays in the scratch array and is not reported.
+ * Scratch needed, with m = n/P and R(v) = v rounded up to a multiple of 256:
+ *   256 + P*(P+1) * (R(m*bits/8) + R(4*m/block) + R(m/block)) bytes,
+ * e.g. 343 KB for P = 4, n = 65536 per rank, INT8, blocks of 128; at most
+ * about 3.2 M elements per rank for P = 4 INT8.  Larger problems return
+ * FC_ERR_TOO_LARGE before anything is launched.
+ * Set-up: the first call on a device (with that device current) looks up the
+ * array's device address with cudaGetSymbolAddress, which may load the
+ * library's module; make that first call before any stream capture.
+ * Every call on a device uses the same array and it keeps the previous
+ * call's contents: two calls whose work overlaps on the GPU (different
+ * streams without ordering between them, or different host threads) race
+ * on it and both results are undefined.  Errors: as for
+ * fc_p2p_allreduce_emulated, plus FC_ERR_TOO_LARGE. */
+#define FC_NOALLOC_SCRATCH_BYTES (16u << 20)
+fc_status fc_p2p_allreduce_emulated_noalloc(int P, fc_dtype dtype, size_t n, int bits, int block,
+                                            const void* const* x, void* const* y, int* status, void* stream);
 
 /* Static description of a status code. */
 const char* fc_status_string(fc_status status);

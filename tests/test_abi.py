@@ -30,7 +30,7 @@ def test_payload_sizes():
 
 
 def test_status_strings():
-    for st in range(5):
+    for st in range(6):
         assert fc.fc_status_string(st)
     assert fc.library().fc_last_cuda_error() == 0
 
@@ -142,3 +142,23 @@ def test_p2p_validation():
     assert call(n=0) == fc.FC_OK
     assert lib.fc_p2p_allreduce(0, 2, 0, 4096, 8, 128, x, y, None, s2, ctr, ctr, 1, st, 0, None) == fc.FC_ERR_INVALID_ARG
     assert lib.fc_p2p_allreduce(0, 2, 0, 4096, 8, 128, x, y, s1, s2, ctr, ctr, 1, None, 0, None) == fc.FC_ERR_INVALID_ARG
+
+
+def test_noalloc_validation_before_any_cuda_call():
+    """The entry point without allocation refuses bad arguments and problems larger than its
+    static scratch on the host, before it looks up the scratch or launches anything."""
+    lib = fc.library()
+
+    def call(P, n, bits=8, block=128, dtype=0, x=XS, y=XS):
+        xp = (ctypes.c_void_p * 8)(*x[:8])
+        yp = (ctypes.c_void_p * 8)(*[a + 0x80000000 for a in y[:8]])
+        return lib.fc_p2p_allreduce_emulated_noalloc(P, dtype, n, bits, block, xp, yp, None, None)
+
+    assert call(4, 0) == fc.FC_OK
+    assert call(3, 3 * 128) == fc.FC_ERR_INVALID_ARG
+    assert call(4, 4 * 128 + 128) == fc.FC_ERR_INVALID_ARG
+    assert call(4, 4 * 128, bits=6) == fc.FC_ERR_INVALID_ARG
+    assert call(4, 4 * 128, dtype=2) == fc.FC_ERR_INVALID_ARG
+    assert lib.fc_p2p_allreduce_emulated_noalloc(4, 0, 512, 8, 128, None, None, None, None) == fc.FC_ERR_INVALID_ARG
+    assert call(4, 4 * 128 * 8192) == fc.FC_ERR_TOO_LARGE            # 4 Mi elements per rank at INT8
+    assert call(8, 1 << 40) == fc.FC_ERR_TOO_LARGE
