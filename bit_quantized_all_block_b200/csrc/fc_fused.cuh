@@ -137,22 +137,25 @@ __device__ __forceinline__ void rank_body(const uint4* raw, const BlockQ& b, flo
     using P2 = Pair<T>;
     using T2 = typename P2::T2;
     const float cqz = __fsub_rn(b.cq, b.zf);   // FC_MAGIC + qmax - z (exact; +inf: no clamp)
+    const float2 inv2 = dup2(b.inv), m2 = dup2(FC_MAGIC), nm2 = dup2(-FC_MAGIC), s2 = dup2(b.s);
     uint32_t words[NC * BITS / 4];
 #pragma unroll
     for (int c = 0; c < NC; c++) {
         const uint32_t w[4] = {raw[c].x, raw[c].y, raw[c].z, raw[c].w};
         float r[8];
 #pragma unroll
-        for (int h = 0; h < 4; h++) {
-            const float2 v = P2::to_f2(as_t2<T2>(w[h]));
-            r[2 * h] = round_product_shifted(v.x, b.inv);       // FC_MAGIC + rne(v*inv)
-            r[2 * h + 1] = round_product_shifted(v.y, b.inv);
-        }
+        for (int h = 0; h < 4; h++)
+            st2(r, 2 * h, fma2(P2::to_f2(as_t2<T2>(w[h])), inv2, m2));   // FC_MAGIC + rne(v*inv)
 #pragma unroll
-        for (int i = 0; i < 8; i++) {
+        for (int i = 0; i < 8; i++)
             r[i] = fminf(r[i], cqz);
-            const float xh = __fmul_rn(__fsub_rn(r[i], FC_MAGIC), b.s);  // (q - z) * s
-            acc[c * 8 + i] = FIRST ? xh : __fadd_rn(acc[c * 8 + i], xh);
+#pragma unroll
+        for (int i = 0; i < 8; i += 2) {
+            const float2 xh = mul2(add2(ld2(r, i), nm2), s2);              // (q - z) * s
+            if (FIRST)
+                st2(acc, c * 8 + i, xh);
+            else
+                acc_add(acc, c * 8 + i, xh);
         }
         if (store)
             pack_shifted<BITS>(r, b, pack_offset<BITS>(b), words, c);
@@ -172,17 +175,21 @@ __device__ __forceinline__ void sum_body(const float* acc, const BlockQ& b, T* y
                                          const QPtr& out, size_t e, bool leader, size_t k)
 {
     const float cqz = __fsub_rn(b.cq, b.zf);
+    const float2 inv2 = dup2(b.inv), m2 = dup2(FC_MAGIC), nm2 = dup2(-FC_MAGIC), s2 = dup2(b.s);
     uint32_t words[NC * BITS / 4];
     uint4 ov[NC];
 #pragma unroll
     for (int c = 0; c < NC; c++) {
         float r[8], o[8];
 #pragma unroll
-        for (int i = 0; i < 8; i++) {
-            r[i] = round_product_shifted(acc[c * 8 + i], b.inv);
+        for (int i = 0; i < 8; i += 2)
+            st2(r, i, fma2(ld2(acc, c * 8 + i), inv2, m2));
+#pragma unroll
+        for (int i = 0; i < 8; i++)
             r[i] = fminf(r[i], cqz);
-            o[i] = __fmul_rn(__fsub_rn(r[i], FC_MAGIC), b.s);
-        }
+#pragma unroll
+        for (int i = 0; i < 8; i += 2)
+            st2(o, i, mul2(add2(ld2(r, i), nm2), s2));
         if constexpr (WIDE)
             ov[c] = narrow8<T>(o);
         else
@@ -241,8 +248,7 @@ __device__ __forceinline__ void rank_body_plain(const uint4* raw, float* acc)
         for (int h = 0; h < 4; h++) {
             const float2 v = P2::to_f2(as_t2<T2>(w[h]));
             const int i = c * 8 + 2 * h;
-            acc[i] = FIRST ? v.x : __fadd_rn(acc[i], v.x);
-            acc[i + 1] = FIRST ? v.y : __fadd_rn(acc[i + 1], v.y);
+            st2(acc, i, FIRST ? v : add2(ld2(acc, i), v));
         }
     }
 }

@@ -108,14 +108,17 @@ __device__ __forceinline__ void quant_store(const float* v, const BlockQ& b, con
 {
     const float cqz = __fsub_rn(b.cq, b.zf);
     const uint32_t offset = pack_offset<BITS>(b);
+    const float2 inv2 = dup2(b.inv), m2 = dup2(FC_MAGIC);
     uint32_t words[NC * BITS / 4];
 #pragma unroll
     for (int c = 0; c < NC; c++) {
         float r[8];
 #pragma unroll
-        for (int i = 0; i < 8; i++) {
-            r[i] = round_product_shifted(v[c * 8 + i], b.inv);
-            if (CLAMP)
+        for (int i = 0; i < 8; i += 2)
+            st2(r, i, fma2(ld2(v, c * 8 + i), inv2, m2));   // FC_MAGIC + rne(v*inv)
+        if (CLAMP) {
+#pragma unroll
+            for (int i = 0; i < 8; i++)
                 r[i] = fminf(r[i], cqz);
         }
         pack_shifted<BITS>(r, b, offset, words, c);
@@ -231,14 +234,18 @@ __global__ void __launch_bounds__(ST_THREADS) k_rs(const RsArgs a)
         float acc[E];
 #pragma unroll
         for (int r = 0; r < P; r++) {
+            const float2 nmz2 = dup2(-mz[r]), s2 = dup2(s[r]);
 #pragma unroll
             for (int c = 0; c < NC; c++) {
                 float sh[8];
                 chunk_shifted<BITS>(w[r], c, sh);
 #pragma unroll
-                for (int i = 0; i < 8; i++) {
-                    const float xh = __fmul_rn(__fsub_rn(sh[i], mz[r]), s[r]);
-                    acc[c * 8 + i] = (r == 0) ? xh : __fadd_rn(acc[c * 8 + i], xh);
+                for (int i = 0; i < 8; i += 2) {
+                    const float2 xh = mul2(add2(ld2(sh, i), nmz2), s2);     // (q - z) * s
+                    if (r == 0)
+                        st2(acc, c * 8 + i, xh);
+                    else
+                        acc_add(acc, c * 8 + i, xh);
                 }
             }
             if (valid_next) {   // refill rank r with the next tile
@@ -293,14 +300,15 @@ __global__ void __launch_bounds__(ST_THREADS) k_ag(const AgArgs a)
             mzn = __uint_as_float(FC_MAGIC_BITS + a.in.zps[en >> lg_block]);
         }
         if (e < a.n) {
+            const float2 nmz2 = dup2(-mz), s2 = dup2(s);
             uint4 ov[NC];
 #pragma unroll
             for (int c = 0; c < NC; c++) {
                 float sh[8], v[8];
                 chunk_shifted<BITS>(w, c, sh);
 #pragma unroll
-                for (int i = 0; i < 8; i++)
-                    v[i] = __fmul_rn(__fsub_rn(sh[i], mz), s);
+                for (int i = 0; i < 8; i += 2)
+                    st2(v, i, mul2(add2(ld2(sh, i), nmz2), s2));
                 ov[c] = narrow8<T>(v);
             }
             store_chunks<NC, WIDE>(y + e, ov);
