@@ -19,11 +19,11 @@
 //  * the P per-rank scale computations of a block are spread over the lanes
 //    of its group (lane r computes rank r) and broadcast with shuffles;
 //  * the upper code clamp binds only when the block maximum's code rounds to
-//    qmax + 1 -- rare -- so it is checked once per block from the maximum;
-//    when no block of the warp needs it, its limit is +inf, so one copy of
-//    each body serves both cases (the rank loop is unrolled P times and its
-//    code size shows up as instruction-fetch stalls); the lower clamp never
-//    binds (see the lower-clamp note in fc_device.cuh);
+//    qmax + 1 -- rare -- so it is checked once per block from the maximum
+//    and applied behind a warp-uniform branch around the per-element minimum
+//    only, so each body exists once (the rank loop is unrolled P times and
+//    its code size shows up as instruction-fetch stalls); the lower clamp
+//    never binds (see the lower-clamp note in fc_device.cuh);
 //    that lane-split form is used whenever a block's thread group has at
 //    least P lanes (SPLIT, chosen by the host from the block size; narrower
 //    groups compute every rank's scale in every lane), so the unrolled loop
@@ -128,15 +128,17 @@ __device__ __forceinline__ void store_thread_codes(uint8_t* codes, size_t e, con
     }
 }
 
-// Step-1 work on one rank's values, chunk by chunk: quantize, dequantize,
-// accumulate in rank order; optionally store codes, scale and zero-point.
+// Step-1 work on one rank's values: quantize, dequantize, accumulate in rank
+// order; optionally store codes, scale and zero-point.  `clamp` (warp-uniform)
+// says whether any block of the warp needs the upper code clamp; the branch
+// skips the per-element minimum in the usual case without a second copy of
+// the body (the rank loop is unrolled P times, so code size matters).
 template <class T, int BITS, int NC, bool FIRST>
-__device__ __forceinline__ void rank_body(const uint4* raw, const BlockQ& b, float* acc, bool store,
+__device__ __forceinline__ void rank_body(const uint4* raw, const BlockQ& b, bool clamp, float* acc, bool store,
                                           const QPtr& out, size_t e, bool leader, size_t k)
 {
     using P2 = Pair<T>;
     using T2 = typename P2::T2;
-    const float cqz = __fsub_rn(b.cq, b.zf);   // FC_MAGIC + qmax - z (exact; +inf: no clamp)
     const float2 inv2 = dup2(b.inv), m2 = dup2(FC_MAGIC), nm2 = dup2(-FC_MAGIC), s2 = dup2(b.s);
     uint32_t words[NC * BITS / 4];
 #pragma unroll
@@ -146,9 +148,12 @@ __device__ __forceinline__ void rank_body(const uint4* raw, const BlockQ& b, flo
 #pragma unroll
         for (int h = 0; h < 4; h++)
             st2(r, 2 * h, fma2(P2::to_f2(as_t2<T2>(w[h])), inv2, m2));   // FC_MAGIC + rne(v*inv)
+        if (clamp) {
+            const float cqz = __fsub_rn(b.cq, b.zf);   // FC_MAGIC + qmax - z (exact)
 #pragma unroll
-        for (int i = 0; i < 8; i++)
-            r[i] = fminf(r[i], cqz);
+            for (int i = 0; i < 8; i++)
+                r[i] = fminf(r[i], cqz);
+        }
 #pragma unroll
         for (int i = 0; i < 8; i += 2) {
             const float2 xh = mul2(add2(ld2(r, i), nm2), s2);              // (q - z) * s
@@ -169,12 +174,12 @@ __device__ __forceinline__ void rank_body(const uint4* raw, const BlockQ& b, flo
     }
 }
 
-// Step 2 on the sums, chunk by chunk: requantize, dequantize, store y (+ payload).
+// Step 2 on the sums: requantize, dequantize, store y (+ payload); `clamp`
+// as for rank_body.
 template <class T, int BITS, int NC, bool WIDE>
-__device__ __forceinline__ void sum_body(const float* acc, const BlockQ& b, T* y, bool store,
+__device__ __forceinline__ void sum_body(const float* acc, const BlockQ& b, bool clamp, T* y, bool store,
                                          const QPtr& out, size_t e, bool leader, size_t k)
 {
-    const float cqz = __fsub_rn(b.cq, b.zf);
     const float2 inv2 = dup2(b.inv), m2 = dup2(FC_MAGIC), nm2 = dup2(-FC_MAGIC), s2 = dup2(b.s);
     uint32_t words[NC * BITS / 4];
     uint4 ov[NC];
@@ -184,9 +189,12 @@ __device__ __forceinline__ void sum_body(const float* acc, const BlockQ& b, T* y
 #pragma unroll
         for (int i = 0; i < 8; i += 2)
             st2(r, i, fma2(ld2(acc, c * 8 + i), inv2, m2));
+        if (clamp) {
+            const float cqz = __fsub_rn(b.cq, b.zf);
 #pragma unroll
-        for (int i = 0; i < 8; i++)
-            r[i] = fminf(r[i], cqz);
+            for (int i = 0; i < 8; i++)
+                r[i] = fminf(r[i], cqz);
+        }
 #pragma unroll
         for (int i = 0; i < 8; i += 2)
             st2(o, i, mul2(add2(ld2(r, i), nm2), s2));
@@ -382,16 +390,10 @@ __global__ void __launch_bounds__(FuShape<P, SMALL>::THREADS, FuShape<P, SMALL>:
                     b = block_q<QB1>(fminf(P2::lo(t), 0.0f), mx);
                     clamp = __any_sync(0xffffffffu, top_code_overflows(mx, b));
                 }
-                // One copy of the rank body per rank (the loop is unrolled P
-                // times, so code size matters): when no block of this warp
-                // needs the upper clamp, its limit is +inf and the clamp is a
-                // no-op instead of a second copy of the body.
-                if (!clamp)
-                    b.cq = __int_as_float(0x7f800000);
                 if (r == 0)
-                    rank_body<T, QB1, NC, true>(raw[r], b, acc, store1, a.step1[r], e, leader, k);
+                    rank_body<T, QB1, NC, true>(raw[r], b, clamp, acc, store1, a.step1[r], e, leader, k);
                 else
-                    rank_body<T, QB1, NC, false>(raw[r], b, acc, store1, a.step1[r], e, leader, k);
+                    rank_body<T, QB1, NC, false>(raw[r], b, clamp, acc, store1, a.step1[r], e, leader, k);
                 if (valid_next)   // refill rank r with the next tile while this one finishes
                     load_chunks<T, NC, WIDE>(raw[r], static_cast<const T*>(a.x[r]) + e + stride);
             }
@@ -419,12 +421,10 @@ __global__ void __launch_bounds__(FuShape<P, SMALL>::THREADS, FuShape<P, SMALL>:
             mx = fmaxf(mx, acc[E - 1]);
             // the next tile's step-1 barrier separates these reads from the next writes
             group_minmax_f32<B1 == 16>(mn, mx, L, red32);
-            BlockQ b2 = block_q<B2>(mn, mx);
+            const BlockQ b2 = block_q<B2>(mn, mx);
             const bool clamp2 = __any_sync(0xffffffffu, top_code_overflows(mx, b2));
-            if (!clamp2)
-                b2.cq = __int_as_float(0x7f800000);   // one body: the clamp is a no-op
             if (valid)
-                sum_body<T, B2, NC, WIDE>(acc, b2, y, a.write_step2 != 0, a.step2, e, leader, k);
+                sum_body<T, B2, NC, WIDE>(acc, b2, clamp2, y, a.write_step2 != 0, a.step2, e, leader, k);
         }
     }
 }

@@ -196,14 +196,15 @@ __global__ void __launch_bounds__(P2P_THREADS) k_p2p(const __grid_constant__ P2P
                 for (int i = 0; i < NW; i++)
                     w[i] = 0;
             }
+            const float2 nmz2 = dup2(-mz), s2 = dup2(s);
 #pragma unroll
             for (int c = 0; c < NC; c++) {
                 float sh[8];
                 chunk_shifted<BITS>(w, c, sh);
 #pragma unroll
-                for (int i = 0; i < 8; i++) {
-                    const float xh = __fmul_rn(__fsub_rn(sh[i], mz), s);
-                    acc[c * 8 + i] = (r == 0) ? xh : __fadd_rn(acc[c * 8 + i], xh);
+                for (int i = 0; i < 8; i += 2) {
+                    const float2 xh = prod2(add2(ld2(sh, i), nmz2), s2);    // (q - z) * s
+                    st2(acc, c * 8 + i, (r == 0) ? xh : add2(ld2(acc, c * 8 + i), xh));
                 }
             }
         }

@@ -241,11 +241,8 @@ __global__ void __launch_bounds__(ST_THREADS) k_rs(const RsArgs a)
                 chunk_shifted<BITS>(w[r], c, sh);
 #pragma unroll
                 for (int i = 0; i < 8; i += 2) {
-                    const float2 xh = mul2(add2(ld2(sh, i), nmz2), s2);     // (q - z) * s
-                    if (r == 0)
-                        st2(acc, c * 8 + i, xh);
-                    else
-                        acc_add(acc, c * 8 + i, xh);
+                    const float2 xh = prod2(add2(ld2(sh, i), nmz2), s2);    // (q - z) * s
+                    st2(acc, c * 8 + i, (r == 0) ? xh : add2(ld2(acc, c * 8 + i), xh));
                 }
             }
             if (valid_next) {   // refill rank r with the next tile
