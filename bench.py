@@ -26,6 +26,7 @@ import argparse
 import datetime
 import hashlib
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -117,7 +118,7 @@ class ClockSampler:
 
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap,clocks.mem")
 
     def __init__(self, index: int):
         self.index = index
@@ -152,7 +153,7 @@ class ClockSampler:
             self.thread.join(timeout=2)
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
+        sm, mx, reasons, power, mem = [], None, set(), [], []
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in self.lines:
             f = [x.strip() for x in line.split(",")]
@@ -163,13 +164,20 @@ class ClockSampler:
                 mx = float(f[2])
             except ValueError:
                 continue
+            try:
+                power.append(float(f[3]))
+                if len(f) > 9:
+                    mem.append(float(f[9]))
+            except ValueError:
+                pass
             for name, val in zip(names, f[5:9]):
                 if val.lower() == "active":
                     reasons.add(name)
         if not sm:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "power_w_max": max(power) if power else None,
+                "mem_mhz": statistics.median(mem) if mem else None}
 
 
 def max_over_ranks(v: float, world: int, device="cuda") -> float:
@@ -570,6 +578,8 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=0,
                     help="token rows per rank for the cpu_baseline sample (0 = the whole workload)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ramp-ms", type=float, default=100.0,
+                    help="untimed device work (ms) enqueued directly before the timed region")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch the timed steps one by one instead of replaying a CUDA graph of them")
     ap.add_argument("--gemm", action="store_true",
@@ -661,9 +671,32 @@ def main():
             torch.cuda.synchronize()
         flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda") if small else None
         ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+        # Clock ramp: starting the clock sampler leaves the GPU idle for a few
+        # hundred ms, and its clocks drop.  Untimed work for at least --ramp-ms of
+        # device time is therefore enqueued directly before the timed region,
+        # with no host synchronisation between the two, so the timed steps run at
+        # the GPU's running clocks however few they are.
+        def unit():
+            if graph is not None:
+                graph.replay()
+            else:
+                if small:
+                    flush.zero_()
+                step()
+        ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ea.record(stream)
+        unit()
+        eb.record(stream)
+        torch.cuda.synchronize()
+        n_ramp = max(1, math.ceil(args.ramp_ms / max(ea.elapsed_time(eb), 1e-3)))
+        ramp_steps = n_ramp * (args.steps if graph is not None else 1)
+
         with ClockSampler(local) as clocks:
             barrier()
             torch.cuda.synchronize()
+            for _ in range(n_ramp):
+                unit()
             if variant == "staged":
                 # events between the stages give each staged kernel its own time
                 marks = []
@@ -764,6 +797,8 @@ def main():
             "config": {"workload": w.name, "description": w.describe(), "variant": variant,
                        "parallelism": f"replicas x{world} (P={w.P} ranks emulated per GPU)",
                        "launch": "CUDA graph of the timed steps" if graph is not None else "stream launches",
+                       "clock_ramp": (f"{ramp_steps} untimed steps (>= {args.ramp_ms:g} ms) enqueued directly before "
+                                      f"the timed region, after the {args.warmup} warm-up steps"),
                        "l2": (f"L2 flushed (512 MB write) before each step, each step timed alone"
                               if small else
                               f"inputs larger than L2 ({in_bytes / 1e6:.0f} MB read per step), no flush")},
