@@ -7,9 +7,10 @@
 // the caller asks for them.  Flash Communication (sciencestack.ai/paper/
 // 2412.04964), TL;DR: the method is implemented as one fused CUDA kernel.
 //
-// The kernel moves ~1 GB per call on the 70B-shaped workload and runs close to
-// both the HBM and the instruction-issue ceilings (about a dozen operations per
-// input element), so it is laid out to cut instructions:
+// The kernel moves ~1 GB per call on the 70B-shaped workload; with about a dozen
+// operations per input element it would be bound by instruction issue as much
+// as by HBM, so it is laid out to cut instructions (after which it waits on
+// its loads rather than on issue):
 //  * thread t of a CTA owns E = 16 contiguous elements of every rank in the
 //    tile (8 in the latency shape); a block of B elements is L = B/E
 //    consecutive threads, so a 128-block needs 8 threads and 3 shuffle
@@ -31,7 +32,10 @@
 //  * each rank's registers are refilled with the next tile's data as soon as
 //    that rank is consumed, so loads stay in flight during the rest of the
 //    tile (software pipelining without extra registers);
-//  * code bytes are formed only when a payload is written.
+//  * code bytes are formed only when a payload is written;
+//  * the per-element floating-point chains run on packed fp32 pairs (see the
+//    contraction note in fc_device.cuh for how the rank-order sum is kept
+//    exact).
 #pragma once
 
 #include "fc_kernels.cuh"
