@@ -172,11 +172,22 @@ class QuantizedAllReduce:
     Collective constructor (every rank, same arguments): allocates this rank's
     arena, exchanges the peer mappings.  Calling the object on this rank's
     partial x (n elements, flat) writes the all-reduced result to y (default: a
-    new tensor) and returns it; every rank receives the same bits."""
+    new tensor) and returns it; every rank receives the same bits.
 
-    def __init__(self, n: int, bits: int, block: int, group=None, ops=None, one_kernel: bool = False):
+    Failures: the host barriers between the steps are monitored with `timeout`
+    seconds; if a rank fails or leaves, the others' call raises RuntimeError
+    within that time (naming the missing rank) instead of blocking.  After such
+    an error the object is unusable; every rank must create a new one."""
+
+    def __init__(self, n: int, bits: int, block: int, group=None, ops=None, one_kernel: bool = False,
+                 timeout: float = 60.0):
+        import datetime
+
         import torch.distributed as dist
         self.dist = dist
+        # a rank that fails or leaves makes the others' next barrier raise after
+        # `timeout` seconds (naming the missing rank) instead of waiting for good
+        self.timeout = datetime.timedelta(seconds=timeout)
         self.group = group if group is not None else dist.group.WORLD
         self.rank = dist.get_rank(self.group)
         self.P = dist.get_world_size(self.group)
@@ -185,7 +196,7 @@ class QuantizedAllReduce:
         backend = dist.get_backend(self.group)
         # host barriers and the handle exchange run on a CPU group
         self.host = self.group if backend == "gloo" else dist.new_group(
-            ranks=dist.get_process_group_ranks(self.group), backend="gloo")
+            ranks=dist.get_process_group_ranks(self.group), backend="gloo", timeout=self.timeout)
         self.bits, self.block = bits, block
         self.layout = Layout(n, self.P, bits, block)
         self.ops = ops if ops is not None else CudaOps()
@@ -206,7 +217,7 @@ class QuantizedAllReduce:
 
     def barrier(self):
         self.ops.sync()
-        self.dist.barrier(group=self.host)
+        self.dist.monitored_barrier(group=self.host, timeout=self.timeout, wait_all_ranks=True)
 
     def __call__(self, x, y=None):
         L, b, B = self.layout, self.bits, self.block

@@ -98,3 +98,51 @@ def test_layout_reserves_aligned_counters():
     assert L.counters % ALIGN == 0 and L.counters + 8 <= L.nbytes
     last = L.step2(0)
     assert L.counters >= last.zps + 2048 // 128
+
+
+def _leaving_rank_main(rank, world, port, out, stall=0.0):
+    """Every rank makes one call; the last rank then leaves (after `stall`
+    seconds alive without taking part), the others call again."""
+    import time
+    from tests.collective_cpu_ops import OracleOps
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    n, dtype, bits, block = world * world * 128 * 2, oracle.FP16, 8, 128
+    ops = OracleOps(dtype)
+    try:
+        ar = QuantizedAllReduce(n, bits, block, ops=ops, timeout=3.0)
+        xs = synth.partials(world, n // block, block, dtype, 0.0, 1.0, seed=5)
+        ar(xs[rank])
+        if rank == world - 1:
+            time.sleep(stall)
+            out[rank] = "left"
+            return
+        t0 = time.time()
+        try:
+            ar(xs[rank])
+            out[rank] = "no error"
+        except RuntimeError as e:
+            out[rank] = ("error", time.time() - t0, str(e)[:200])
+    finally:
+        ops.close()          # this rank's arena and its views of the others' (no collective step)
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("stall", [0.0, 8.0], ids=["exits", "stalls"])
+def test_a_rank_that_leaves_ends_the_others_call_with_an_error(stall):
+    """Failure detection on the host: after one call the last rank leaves --
+    at once (its connections close) or after staying alive 8 s without taking
+    part; the others' next call must end with an error, at the latest after
+    the collective's 3 s timeout, never waiting for the missing rank."""
+    world = 3
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    mp.start_processes(_leaving_rank_main, args=(world, _free_port(), out, stall), nprocs=world, join=True,
+                       start_method="spawn")
+    assert out[world - 1] == "left"
+    for r in range(world - 1):
+        res = out[r]
+        assert res[0] == "error", f"rank {r}: {res}"
+        assert res[1] < (6.0 if stall else 30.0), f"rank {r} waited {res[1]:.1f} s"
+    if stall:
+        assert any(2.5 < out[r][1] for r in range(world - 1)), "the timeout path was not taken"
