@@ -19,6 +19,11 @@ over all GPUs.
 
 ``--impl reference`` times the CPU oracle (the plain definition the kernels
 are checked against) on a bounded sample of the same workload, on rank 0.
+
+Before every timed region, untimed steps worth ``--ramp-ms`` (default 100 ms)
+of device time are enqueued directly ahead of it, with no host
+synchronisation in between, so that however few steps are timed they run at
+the GPU's running clocks (starting the clock sampler leaves the GPU idle).
 """
 from __future__ import annotations
 
