@@ -765,6 +765,48 @@ def main():
         def e2e_zero_copy():
             step(xs_pinned, y_host)
 
+        # Pipelined: token-row chunks (each an all-reduce of its own, every block
+        # lying in one chunk) on three streams, so the H2D copy of chunk c + 1,
+        # the fused call on chunk c and the D2H copy of chunk c - 1 overlap.
+        unit = w.H * (w.P * w.block) // math.gcd(w.H, w.P * w.block)
+        nchunks = min(8, w.n // unit) if variant.startswith("fused") else 0
+        bounds = []
+        if nchunks > 1:
+            per = (w.n // unit // nchunks) * unit
+            bounds = [(c * per, (c + 1) * per if c + 1 < nchunks else w.n) for c in range(nchunks)]
+        s_in, s_cmp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+
+        def qslice(q, e0, e1):
+            return fc.QBuf(q.codes[e0 * w.bits // 8:e1 * w.bits // 8], q.scales[e0 // w.block:e1 // w.block],
+                           q.zps[e0 // w.block:e1 // w.block], e1 - e0, w.bits, w.block)
+
+        def e2e_pipelined():
+            start = torch.cuda.Event()
+            start.record(stream)
+            for st in (s_in, s_cmp, s_out):
+                st.wait_event(start)
+            for e0, e1 in bounds:
+                with torch.cuda.stream(s_in):
+                    for r in range(w.P):
+                        xs[r][e0:e1].copy_(xs_pinned[r][e0:e1], non_blocking=True)
+                ev_in = torch.cuda.Event()
+                ev_in.record(s_in)
+                s_cmp.wait_event(ev_in)
+                if variant == "fused":
+                    fc.fc_quantized_allreduce([x[e0:e1] for x in xs], w.bits, w.block, y=y[e0:e1],
+                                              step1=[qslice(q, e0, e1) for q in s1], step2=qslice(s2, e0, e1),
+                                              stream=s_cmp)
+                else:
+                    fc.fc_quantized_allreduce([x[e0:e1] for x in xs], w.bits, w.block, y=y[e0:e1], stream=s_cmp)
+                ev_cmp = torch.cuda.Event()
+                ev_cmp.record(s_cmp)
+                s_out.wait_event(ev_cmp)
+                with torch.cuda.stream(s_out):
+                    y_host[e0:e1].copy_(y[e0:e1], non_blocking=True)
+            end = torch.cuda.Event()
+            end.record(s_out)
+            stream.wait_event(end)
+
         def time_e2e(fn):
             for _ in range(2):
                 fn()
@@ -779,11 +821,22 @@ def main():
             return max_over_ranks(a.elapsed_time(b) / args.e2e_steps, world)
 
         ms_copies = time_e2e(e2e_copies)
+        y_dev = y.view(torch.int16).cpu()          # the device-buffer call's output
         ms_zero = time_e2e(e2e_zero_copy)
-        e2e_exact = bool(torch.equal(y_host.view(torch.int16), y.view(torch.int16).cpu()))
-        # the headline e2e figure is the faster of the two ways a user can call the library
-        zero_wins = ms_zero <= ms_copies
-        ms_e2e = ms_zero if zero_wins else ms_copies
+        e2e_exact = bool(torch.equal(y_host.view(torch.int16), y_dev))
+        ms_pipe, pipe_exact = None, None
+        if bounds:
+            y_host.zero_()
+            ms_pipe = time_e2e(e2e_pipelined)
+            pipe_exact = bool(torch.equal(y_host.view(torch.int16), y_dev))
+        # the headline e2e figure is the fastest of the ways a user can call the library on host buffers
+        forms = {"zero-copy: the call on page-locked host buffers": ms_zero,
+                 "explicit copies: H2D of the inputs, the call on device buffers, D2H of the result": ms_copies}
+        if ms_pipe is not None:
+            forms[f"pipelined: {len(bounds)} token-row chunks, H2D / fused call / D2H overlapped on three "
+                  f"streams"] = ms_pipe
+        e2e_mode = min(forms, key=forms.get)
+        ms_e2e = forms[e2e_mode]
 
         in_bytes = w.P * w.n * 2
         value = job_throughput(in_bytes, world, ms)
@@ -813,11 +866,13 @@ def main():
                          "algorithmic_bytes_per_launch": alg if variant.startswith("fused") else None,
                          "algorithmic_bytes_per_step": alg},
             "e2e": {"value": round(value_e2e, 3), "unit": "GB/s", "h2d_bytes_per_step": in_bytes,
-                    "mode": ("zero-copy: the call on page-locked host buffers" if zero_wins else
-                             "explicit copies: H2D of the inputs, the call on device buffers, D2H of the result"),
+                    "mode": e2e_mode,
                     "zero_copy_value": round(job_throughput(in_bytes, world, ms_zero), 3),
                     "explicit_copies_value": round(job_throughput(in_bytes, world, ms_copies), 3),
+                    "pipelined_value": (round(job_throughput(in_bytes, world, ms_pipe), 3)
+                                        if ms_pipe is not None else None),
                     "zero_copy_output_equals_device_path": e2e_exact,
+                    "pipelined_output_equals_device_path": pipe_exact,
                     "d2h_bytes_per_step": w.n * 2},
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clocks.summary(),
