@@ -162,3 +162,33 @@ def test_noalloc_validation_before_any_cuda_call():
     assert lib.fc_p2p_allreduce_emulated_noalloc(4, 0, 512, 8, 128, None, None, None, None) == fc.FC_ERR_INVALID_ARG
     assert call(4, 4 * 128 * 8192) == fc.FC_ERR_TOO_LARGE            # 4 Mi elements per rank at INT8
     assert call(8, 1 << 40) == fc.FC_ERR_TOO_LARGE
+
+
+def _prototypes():
+    """{name: [parameter declarations]} for every function include/fc.h declares."""
+    import re
+    text = open(fc.HEADER_PATH).read()
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    protos = {}
+    for m in re.finditer(r"(?:fc_status|const char\*|int)\s+(fc_\w+)\s*\(([^)]*)\)\s*;", text):
+        params = [p.strip() for p in m.group(2).split(",") if p.strip() and p.strip() != "void"]
+        protos[m.group(1)] = params
+    return protos
+
+
+def test_binding_signatures_match_the_header():
+    """Every ctypes signature the binding sets has the header's arity, and each
+    argument is a pointer exactly where the header declares one."""
+    protos = _prototypes()
+    assert set(protos) == set(fc.declared_symbols())
+    lib = fc.library()
+    pointer_types = (ctypes.c_void_p, ctypes.c_char_p)
+    for name, params in protos.items():
+        argtypes = getattr(lib, name).argtypes
+        if argtypes is None:
+            continue
+        assert len(argtypes) == len(params), f"{name}: {len(argtypes)} ctypes arguments, header has {len(params)}"
+        for decl, t in zip(params, argtypes):
+            is_ptr = "*" in decl
+            t_ptr = t in pointer_types or hasattr(t, "_type_") and issubclass(t, ctypes._Pointer)
+            assert is_ptr == bool(t_ptr), f"{name}: '{decl}' bound as {t}"
