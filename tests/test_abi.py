@@ -192,3 +192,47 @@ def test_binding_signatures_match_the_header():
             is_ptr = "*" in decl
             t_ptr = t in pointer_types or hasattr(t, "_type_") and issubclass(t, ctypes._Pointer)
             assert is_ptr == bool(t_ptr), f"{name}: '{decl}' bound as {t}"
+
+
+def test_gemm_validation():
+    """fc_gemm_quantize refuses bad shapes, block sizes, missing or misaligned buffers and
+    outputs that overlap the operands -- all before any CUDA call."""
+    lib = fc.library()
+    a, w, part, st = A, A + 0x8000000, A + 0x10000000, A + 0x18000000
+    out = qb(A + 0x20000000)
+
+    def call(M=256, N=512, K=128, bits=8, block=128, a=a, w=w, out=out, part=part, st=st, dtype=0):
+        return lib.fc_gemm_quantize(ctypes.c_void_p(a), ctypes.c_void_p(w), dtype, M, N, K, bits, block,
+                                    ctypes.byref(out) if out is not None else None, ctypes.c_void_p(part)
+                                    if part is not None else None, ctypes.c_void_p(st) if st is not None else None,
+                                    None)
+
+    for kw in (dict(M=100), dict(N=100), dict(K=100), dict(M=0), dict(block=256), dict(block=16),
+               dict(bits=5), dict(dtype=2), dict(out=None, part=None), dict(st=None), dict(a=0)):
+        assert call(**kw) == fc.FC_ERR_INVALID_ARG, kw
+    assert call(a=a + 8) == fc.FC_ERR_MISALIGNED
+    assert call(part=part + 4) == fc.FC_ERR_MISALIGNED
+    assert call(st=st + 2) == fc.FC_ERR_MISALIGNED
+    assert call(part=a + 0x1000) == fc.FC_ERR_INVALID_ARG          # partial overlaps a
+    assert call(st=w) == fc.FC_ERR_INVALID_ARG                     # status overlaps w
+
+
+def test_per_step_width_validation():
+    """fc_quantized_allreduce_ex: widths outside {4, 8, 16}, a payload for an unquantized step,
+    sizes that are not whole chunks, and the width combinations this build does not provide."""
+    lib = fc.library()
+
+    def call(P=4, n=4096, b1=8, b2=4, block=128, step1=None, step2=None):
+        xp = (ctypes.c_void_p * P)(*XS[:P])
+        s1 = (fc.fc_qbuf * P)(*step1) if step1 is not None else None
+        return lib.fc_quantized_allreduce_ex(xp, P, 0, n, b1, b2, block, ctypes.c_void_p(A + 0x40000000), s1,
+                                             ctypes.byref(step2) if step2 is not None else None, None)
+
+    assert call(b1=5) == fc.FC_ERR_INVALID_ARG
+    assert call(b2=12) == fc.FC_ERR_INVALID_ARG
+    assert call(b1=16, step1=[qb(A + 0x50000000 + i * 0x4000000) for i in range(4)]) == fc.FC_ERR_INVALID_ARG
+    assert call(b2=16, step2=qb(A + 0x60000000)) == fc.FC_ERR_INVALID_ARG
+    assert call(n=4096 + 128) == fc.FC_ERR_INVALID_ARG
+    assert call(P=3, n=3 * 128 * 4, b1=8, b2=4) == fc.FC_ERR_UNSUPPORTED
+    assert call(P=3, n=3 * 128 * 4, b1=16, b2=16) == fc.FC_ERR_UNSUPPORTED
+    assert call(n=0) == fc.FC_OK
