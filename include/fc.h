@@ -75,7 +75,7 @@ extern "C" {
 typedef enum {
     FC_OK = 0,
     FC_ERR_INVALID_ARG = 1, /* bad size, bits, block, P, NULL or overlapping buffers */
-    FC_ERR_UNSUPPORTED = 2, /* a combination this build does not provide          */
+    FC_ERR_UNSUPPORTED = 2, /* a combination the library does not provide         */
     FC_ERR_MISALIGNED = 3,  /* a device pointer is not 16-byte aligned             */
     FC_ERR_CUDA = 4,        /* a CUDA call failed; see fc_last_cuda_error()       */
     FC_ERR_TOO_LARGE = 5    /* needs more than the library's fixed scratch memory */

@@ -219,7 +219,7 @@ def test_gemm_validation():
 
 def test_per_step_width_validation():
     """fc_quantized_allreduce_ex: widths outside {4, 8, 16}, a payload for an unquantized step,
-    sizes that are not whole chunks, and the width combinations this build does not provide."""
+    sizes that are not whole chunks, and the width combinations the library does not provide."""
     lib = fc.library()
 
     def call(P=4, n=4096, b1=8, b2=4, block=128, step1=None, step2=None):
