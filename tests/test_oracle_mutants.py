@@ -37,6 +37,8 @@ MUTANTS = {
     "symmetric_range": ("float d = mx - mn;", "float d = 2.0f * fmaxf(mx, -mn);"),
     "output_truncated": ("double kr = nearbyint(k);", "double kr = floor(k);"),
     "zero_block_scale_zero": ("(d == 0.0f) ? 1.0f :", "(d == 0.0f) ? 0.0f :"),
+    # the doubly rounded reading: the product rounded to fp32, then to an integer
+    "product_rounded_to_fp32_first": ("double t = (double)a * (double)b;", "double t = (double)(float)(a * b);"),
 }
 
 
@@ -47,6 +49,7 @@ def battery():
         for bits in (8, 4):
             bf.test_quantize_bruteforce(dt, bits)
             bf.test_allreduce_bruteforce(dt, bits)
+            bf.test_codes_round_the_exact_product(dt, bits)
             inv.test_grid_round_trip(dt, bits)
             inv.test_allreduce_error_bound(dt, bits)
     cv.test_narrow_fp16_vs_numpy()
