@@ -7,6 +7,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cstring>
 #include <map>
 #include <mutex>
@@ -65,15 +66,41 @@ fc_status check_qbuf(const fc_qbuf* q, size_t n, int bits, int block, Range* out
     return FC_OK;
 }
 
+// Whether an output range overlaps another output or an input (inputs may
+// overlap each other).  Sort by start and sweep: of two ranges, the one that
+// starts later overlaps the other iff it starts before that one ends, so each
+// range is checked against the furthest end seen so far among outputs (and,
+// for an output, among all ranges).  Up to kMaxRanges non-empty ranges; more
+// are refused as if they overlapped (no caller comes near it).
+constexpr int kMaxRanges = 512;
+
 bool any_overlap(const Range* outs, int nout, const Range* ins, int nin)
 {
-    for (int i = 0; i < nout; i++) {
-        for (int j = 0; j < nin; j++)
-            if (overlap(outs[i], ins[j]))
+    struct Tagged {
+        uintptr_t b, e;
+        bool out;
+    } r[kMaxRanges];
+    int k = 0;
+    for (int pass = 0; pass < 2; pass++) {
+        const Range* src = pass == 0 ? outs : ins;
+        const int cnt = pass == 0 ? nout : nin;
+        for (int i = 0; i < cnt; i++) {
+            if (src[i].len == 0)
+                continue;
+            if (k == kMaxRanges)
                 return true;
-        for (int j = i + 1; j < nout; j++)
-            if (overlap(outs[i], outs[j]))
-                return true;
+            const uintptr_t b = reinterpret_cast<uintptr_t>(src[i].p);
+            r[k++] = {b, b + src[i].len, pass == 0};
+        }
+    }
+    std::sort(r, r + k, [](const Tagged& a, const Tagged& b) { return a.b < b.b; });
+    uintptr_t end_out = 0, end_any = 0;
+    for (int i = 0; i < k; i++) {
+        if (r[i].b < (r[i].out ? end_any : end_out))
+            return true;
+        end_any = r[i].e > end_any ? r[i].e : end_any;
+        if (r[i].out)
+            end_out = r[i].e > end_out ? r[i].e : end_out;
     }
     return false;
 }
@@ -517,27 +544,41 @@ fc_status p2p_common(bool emu, int rank, int P, fc_dtype dtype, size_t n, int bi
         a.x[i] = x[i];
         a.y[i] = y[i];
     }
-    Range scratch[3];
+    // every buffer the kernel writes (outputs, payloads, counters, status)
+    // must not overlap another one or an input
+    Range outs[fc::FC_MAX_P * (1 + 3 * fc::FC_MAX_P + 3 + 2) + 1], ins[fc::FC_MAX_P];
+    int nout = 0;
+    for (int i = 0; i < nio; i++) {
+        outs[nout++] = {y[i], n * 2};
+        ins[i] = {x[i], n * 2};
+    }
     for (int p = 0; p < P; p++) {
         for (int c = 0; c < P; c++) {
-            fc_status st = check_qbuf(&s1[p * P + c], m, bits, block, scratch);
+            fc_status st = check_qbuf(&s1[p * P + c], m, bits, block, outs + nout);
             if (st != FC_OK)
                 return st;
+            nout += 3;
             a.s1[p][c] = qptr(&s1[p * P + c]);
         }
-        fc_status st = check_qbuf(&s2[p], m, bits, block, scratch);
+        fc_status st = check_qbuf(&s2[p], m, bits, block, outs + nout);
         if (st != FC_OK)
             return st;
+        nout += 3;
         a.s2[p] = qptr(&s2[p]);
         if (ctr1[p] == nullptr || ctr2[p] == nullptr)
             return FC_ERR_INVALID_ARG;
         if ((reinterpret_cast<uintptr_t>(ctr1[p]) & 3u) || (reinterpret_cast<uintptr_t>(ctr2[p]) & 3u))
             return FC_ERR_MISALIGNED;
+        outs[nout++] = {ctr1[p], sizeof(unsigned int)};
+        outs[nout++] = {ctr2[p], sizeof(unsigned int)};
         a.ctr1[p] = ctr1[p];
         a.ctr2[p] = ctr2[p];
     }
     if (reinterpret_cast<uintptr_t>(status) & 3u)
         return FC_ERR_MISALIGNED;
+    outs[nout++] = {status, sizeof(int)};
+    if (any_overlap(outs, nout, ins, nio))
+        return FC_ERR_INVALID_ARG;
     a.status = status;
     a.m = m;
     a.block = block;
@@ -733,11 +774,41 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[FC_NOALLOC_SCRA
 constexpr size_t kNoallocHeader = 256;
 constexpr int kNoallocMaxDevices = 64;
 std::mutex g_noalloc_mu;
-unsigned char* g_noalloc_addr[kNoallocMaxDevices];   // device address of the array, per device
+unsigned char* g_noalloc_addr[kNoallocMaxDevices];        // device address of the array, per device
+unsigned long long g_noalloc_ctx[kNoallocMaxDevices];     // id of the context that address belongs to
 
 size_t round256(size_t v) { return (v + 255) & ~(size_t)255; }
 
-// Device address of the scratch array on the current device (looked up once per device).
+// Unique id of the current CUDA context (ids are never reused within a
+// process, so a context created after a reset of the device has a new one);
+// false when no context is current or the driver lacks the query.
+bool current_context_id(unsigned long long* id)
+{
+    using GetCurrent = CUresult (*)(CUcontext*);
+    using GetId = CUresult (*)(CUcontext, unsigned long long*);
+    static GetCurrent get_current = nullptr;
+    static GetId get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<GetCurrent>(p);
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<GetId>(p);
+    });
+    CUcontext ctx = nullptr;
+    if (get_current == nullptr || get_id == nullptr || get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr)
+        return false;
+    return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+// Device address of the scratch array on the current device: looked up with
+// cudaGetSymbolAddress once per device, and again whenever the device's
+// context is not the one the address was looked up in (after a reset of the
+// device the module, and with it the array, can be loaded at a new address).
 fc_status noalloc_scratch(unsigned char** out)
 {
     int dev = 0;
@@ -746,13 +817,17 @@ fc_status noalloc_scratch(unsigned char** out)
         return cuda_fail(e);
     if (dev < 0 || dev >= kNoallocMaxDevices)
         return FC_ERR_UNSUPPORTED;
+    unsigned long long ctx = 0;
+    const bool known = current_context_id(&ctx);
     std::lock_guard<std::mutex> lock(g_noalloc_mu);
-    if (g_noalloc_addr[dev] == nullptr) {
+    if (g_noalloc_addr[dev] == nullptr || !known || g_noalloc_ctx[dev] != ctx) {
         void* ptr = nullptr;
         e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
         if (e != cudaSuccess)
             return cuda_fail(e);
+        // the lookup may have created the context: take its id now
         g_noalloc_addr[dev] = static_cast<unsigned char*>(ptr);
+        g_noalloc_ctx[dev] = current_context_id(&ctx) ? ctx : 0;
     }
     *out = g_noalloc_addr[dev];
     return FC_OK;

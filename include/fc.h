@@ -241,7 +241,9 @@ fc_status fc_ipc_close(void* base);
  * The kernel is launched cooperatively (its CTAs wait on each other and on the
  * peers'): no other kernel that waits on this rank may share the GPU.  Requires
  * n % (P*block) == 0, 16-byte-aligned payloads, 4-byte-aligned counters.  The
- * ranks' calls must use the same n, bits, block, dtype and epoch. */
+ * buffers the kernel writes or counts on (y, every payload, every counter, the
+ * status word) must not overlap one another or x: FC_ERR_INVALID_ARG before
+ * launch.  The ranks' calls must use the same n, bits, block, dtype and epoch. */
 fc_status fc_p2p_allreduce(int rank, int P, fc_dtype dtype, size_t n, int bits, int block, const void* x, void* y,
                            const fc_qbuf* s1, const fc_qbuf* s2, unsigned int* const* ctr1,
                            unsigned int* const* ctr2, unsigned int epoch, int* status, int ctas_per_rank,
@@ -283,7 +285,9 @@ fc_status fc_p2p_allreduce_emulated(int P, fc_dtype dtype, size_t n, int bits, i
  *                                    P device pointers; n per rank);
  *   status   device int, or NULL: set to 0 on the stream, OR-ed with 1 if a
  *            wait inside the kernel gave up (outputs then invalid).  With
- *            NULL that flag stays in the scratch array and is not reported.
+ *            NULL that flag stays in the scratch array and nothing reports
+ *            it: the call still returns FC_OK.  A caller that must detect a
+ *            wait that gave up passes a status word.
  * Scratch needed, with m = n/P and R(v) = v rounded up to a multiple of 256:
  *   256 + P*(P+1) * (R(m*bits/8) + R(4*m/block) + R(m/block)) bytes,
  * e.g. 343 KB for P = 4, n = 65536 per rank, INT8, blocks of 128; at most
@@ -291,7 +295,11 @@ fc_status fc_p2p_allreduce_emulated(int P, fc_dtype dtype, size_t n, int bits, i
  * FC_ERR_TOO_LARGE before anything is launched.
  * Set-up: the first call on a device (with that device current) looks up the
  * array's device address with cudaGetSymbolAddress, which may load the
- * library's module; make that first call before any stream capture.
+ * library's module; make that first call before any stream capture.  Later
+ * calls reuse the address while the device's CUDA context is the same one (by
+ * its unique context id); the first call after the context was destroyed and
+ * re-created (cudaDeviceReset) looks the address up again, so it too belongs
+ * before any capture.
  * Every call on a device uses the same array and it keeps the previous
  * call's contents: two calls whose work overlaps on the GPU (different
  * streams without ordering between them, or different host threads) race

@@ -144,6 +144,43 @@ def test_p2p_validation():
     assert lib.fc_p2p_allreduce(0, 2, 0, 4096, 8, 128, x, y, s1, s2, ctr, ctr, 1, None, 0, None) == fc.FC_ERR_INVALID_ARG
 
 
+def test_p2p_overlap_validation():
+    """Buffers the one-kernel all-reduce writes may not overlap each other or its input."""
+    lib = fc.library()
+    P = 2
+    ctr1 = (ctypes.c_void_p * 2)(A + 0x70000000, A + 0x70000010)
+    ctr2 = (ctypes.c_void_p * 2)(A + 0x70000020, A + 0x70000030)
+    x, y = A + 0x60000000, A + 0x68000000
+
+    def call(s1_bases=None, s2_bases=None, st=A + 0x70000100, yy=y, c2=ctr2, emu=False):
+        s1 = (fc.fc_qbuf * 4)(*[qb(b) for b in (s1_bases or [A + i * 0x100000 for i in range(4)])])
+        s2 = (fc.fc_qbuf * 2)(*[qb(b) for b in (s2_bases or [A + 0x400000 + i * 0x100000 for i in range(2)])])
+        if emu:
+            xp = (ctypes.c_void_p * 2)(x, x + 0x10000)
+            yp = (ctypes.c_void_p * 2)(yy, yy + 0x10000)
+            return lib.fc_p2p_allreduce_emulated(P, 0, 4096, 8, 128, xp, yp, s1, s2, ctr1, c2, 1,
+                                                 ctypes.c_void_p(st), 0, None)
+        return lib.fc_p2p_allreduce(0, P, 0, 4096, 8, 128, ctypes.c_void_p(x), ctypes.c_void_p(yy), s1, s2,
+                                    ctr1, c2, 1, ctypes.c_void_p(st), 0, None)
+
+    for emu in (False, True):
+        # two step-1 payloads share their codes
+        assert call(s1_bases=[A, A, A + 0x200000, A + 0x300000], emu=emu) == fc.FC_ERR_INVALID_ARG
+        # a step-2 payload's codes inside a step-1 payload's codes
+        assert call(s2_bases=[A + 0x100, A + 0x500000], emu=emu) == fc.FC_ERR_INVALID_ARG
+        # the output over the input, the status word on a counter, a counter on a counter
+        assert call(yy=x + 0x100, emu=emu) == fc.FC_ERR_INVALID_ARG
+        assert call(st=A + 0x70000010, emu=emu) == fc.FC_ERR_INVALID_ARG
+        assert call(c2=(ctypes.c_void_p * 2)(A + 0x70000000, A + 0x70000030), emu=emu) == fc.FC_ERR_INVALID_ARG
+    # emulated: one rank's output over another rank's output
+    xp = (ctypes.c_void_p * 2)(x, x + 0x10000)
+    yp = (ctypes.c_void_p * 2)(y, y + 0x100)
+    s1 = (fc.fc_qbuf * 4)(*[qb(A + i * 0x100000) for i in range(4)])
+    s2 = (fc.fc_qbuf * 2)(*[qb(A + 0x400000 + i * 0x100000) for i in range(2)])
+    assert lib.fc_p2p_allreduce_emulated(P, 0, 4096, 8, 128, xp, yp, s1, s2, ctr1, ctr2, 1,
+                                         ctypes.c_void_p(A + 0x70000100), 0, None) == fc.FC_ERR_INVALID_ARG
+
+
 def test_noalloc_validation_before_any_cuda_call():
     """The entry point without allocation refuses bad arguments and problems larger than its
     static scratch on the host, before it looks up the scratch or launches anything."""

@@ -8,11 +8,12 @@ caching allocator.  fc_p2p_allreduce_emulated_noalloc serves them: it keeps the
 wire payloads, the phase counters and the status word in the library's own
 static device array, and the caller passes only inputs and outputs.
 
-Checked here through the C ABI (ctypes on libfc.so): two calls in a row on the
-same scratch give the same bits as fc_p2p_allreduce_emulated with caller-owned
-scratch (stale payloads or counters from the first call would show in the
-second); the largest problem that fits the array runs and one more chunk of
-blocks is refused before any launch.  This file is collected last so that a run
+Checked here through the C ABI (ctypes on libfc.so): on two calls in a row on
+the same scratch every rank's output equals the CPU oracle's all-reduce of the
+same inputs, bit for bit, and the bits of fc_p2p_allreduce_emulated with
+caller-owned scratch (stale payloads or counters from the first call would
+show in the second); the largest problem that fits the array runs and one more
+chunk of blocks is refused before any launch.  This file is collected last so that a run
 stopping at its first failure has run every other test before it."""
 import ctypes
 
@@ -56,6 +57,15 @@ def _with_caller_scratch(xs, bits, block):
     return [host_u16(y) for y in ys]
 
 
+def _check_against_oracle(xs_host, ys, dtype, bits, block, what):
+    """Every rank's output equals the oracle's all-reduce of the host inputs."""
+    y_ref = oracle.allreduce(list(xs_host), dtype, bits, block)[0]
+    for p, y in enumerate(ys):
+        got = host_u16(y)
+        bad = np.nonzero(got != y_ref)[0]
+        assert bad.size == 0, f"{what}, rank {p}: {bad.size} outputs differ from the oracle, first at {bad[:8]}"
+
+
 def _scratch_bytes(P, n, bits, block):
     r = lambda v: (v + 255) // 256 * 256
     m = n // P
@@ -70,11 +80,13 @@ def _scratch_bytes(P, n, bits, block):
 def test_two_calls_in_a_row_match_the_allocating_entry_point(P, bits, block, dtype, n):
     status = torch.full((1,), -1, dtype=torch.int32, device="cuda")
     for seed in (70, 71):                       # the second call reuses the first call's scratch
-        xs = to_dev(synth.partials(P, n // block, block, dtype, 0.05, 20.0, seed=seed + P), dtype)
+        xh = synth.partials(P, n // block, block, dtype, 0.05, 20.0, seed=seed + P)
+        xs = to_dev(xh, dtype)
         ys = [torch.full_like(x, float("nan")) for x in xs]
         assert _noalloc(xs, ys, bits, block, status) == fc.FC_OK
         torch.cuda.synchronize()
         assert int(status.item()) == 0
+        _check_against_oracle(xh, ys, dtype, bits, block, f"call with seed {seed}")
         want = _with_caller_scratch(xs, bits, block)
         for p in range(P):
             assert np.array_equal(host_u16(ys[p]), want[p]), f"call with seed {seed}, rank {p}: output differs"
@@ -83,10 +95,12 @@ def test_two_calls_in_a_row_match_the_allocating_entry_point(P, bits, block, dty
 def test_without_a_status_word():
     P, bits, block, dtype, n = 4, 4, 128, oracle.FP16, 4 * 128 * 9
     for seed in (72, 73):
-        xs = to_dev(synth.partials(P, n // block, block, dtype, 0.0, 1.0, seed=seed), dtype)
+        xh = synth.partials(P, n // block, block, dtype, 0.0, 1.0, seed=seed)
+        xs = to_dev(xh, dtype)
         ys = [torch.empty_like(x) for x in xs]
         assert _noalloc(xs, ys, bits, block, None) == fc.FC_OK
         torch.cuda.synchronize()
+        _check_against_oracle(xh, ys, dtype, bits, block, f"seed {seed}")
         want = _with_caller_scratch(xs, bits, block)
         for p in range(P):
             assert np.array_equal(host_u16(ys[p]), want[p])
@@ -101,11 +115,13 @@ def test_the_largest_problem_that_fits_and_one_chunk_more():
     assert _scratch_bytes(P, n, bits, block) > fc.FC_NOALLOC_SCRATCH_BYTES - 32 * 1024   # the array's far end is used
     status = torch.full((1,), -1, dtype=torch.int32, device="cuda")
     for seed in (74, 75):
-        xs = to_dev(synth.partials(P, n // block, block, dtype, 0.001, 50.0, seed=seed), dtype)
+        xh = synth.partials(P, n // block, block, dtype, 0.001, 50.0, seed=seed)
+        xs = to_dev(xh, dtype)
         ys = [torch.empty_like(x) for x in xs]
         assert _noalloc(xs, ys, bits, block, status) == fc.FC_OK
         torch.cuda.synchronize()
         assert int(status.item()) == 0
+        _check_against_oracle(xh, ys, dtype, bits, block, f"seed {seed}")
         want = _with_caller_scratch(xs, bits, block)
         for p in range(P):
             assert np.array_equal(host_u16(ys[p]), want[p]), f"seed {seed}, rank {p}: output differs"
