@@ -568,6 +568,208 @@ def run_message_sweep(args):
             torch.cuda.empty_cache()
 
 
+# ---- the P-GPU exchange against NCCL (one process per GPU) ----------------------
+# Flash Communication (sciencestack.ai/paper/2412.04964), Abstract and Fig. 1:
+# the quantized two-step all-reduce against NCCL's fp16 ring all-reduce of the
+# same partial, over the message range of decode to prefill.  The sweep logic
+# is backend-neutral (`collective_sweep`); `CudaCollectiveEnv` is the GPU form
+# run under torchrun, and the CPU tests drive the same function with gloo ranks.
+
+COLLECTIVE_BLOCK = 128
+
+
+def collective_points(P: int, block: int = COLLECTIVE_BLOCK, min_bytes: int = 16 << 10, max_bytes: int = 1 << 30):
+    """(bits, elements per rank) of the sweep: fp16 messages of 16 KB .. 1 GB
+    per rank in powers of two, INT8 then INT4, each rounded down to whole
+    chunks of blocks (a multiple of P * block elements)."""
+    sizes = []
+    b = min_bytes
+    while b <= max_bytes:
+        n = (b // 2) // (P * block) * (P * block)
+        if n > 0:
+            sizes.append(n)
+        b *= 2
+    return [(bits, n) for bits in (8, 4) for n in sizes]
+
+
+def wire_bytes_per_rank(P: int, n: int, bits: int, block: int) -> dict:
+    """Bytes each rank receives per call: the quantized exchange pulls (P-1)/P
+    of a payload in the reduce-scatter and again in the all-gather; NCCL's
+    ring all-reduce moves 2 (P-1)/P of the fp16 message."""
+    w2 = n * bits // 8 + 5 * (n // block)
+    return {"quantized": 2 * (P - 1) * w2 // P, "nccl_fp16_ring": 2 * (P - 1) * 2 * n // P}
+
+
+def collective_sweep(env, points, steps: int, warmup: int, emit, block: int = COLLECTIVE_BLOCK):
+    """Time every form of the P-rank quantized all-reduce and the baseline
+    all-reduce at each point; emit one dict per point (on rank 0).
+
+    env supplies: rank, world, forms (names -> one_kernel flag; the one-kernel
+    form only where each rank has its own GPU), partial(n) (this rank's seeded
+    partial), expected(n, bits, block) (this rank's output of the one-GPU fused
+    all-reduce of all P partials), allreduce(n, bits, block, one_kernel) (a
+    QuantizedAllReduce), new_output(x), equal(a, b), baseline_buffer(x) and
+    baseline(buf) (one fp16 all-reduce of the message), timed(fn) (elapsed ms
+    of fn's work on this rank's device), barrier(), all_true(flag) and
+    max_over_ranks(v).  Every rank runs the same collective calls in the same
+    order."""
+    P = env.world
+    for bits, n in points:
+        x = env.partial(n)
+        want = env.expected(n, bits, block)
+        us, exact, status = {}, {}, {}
+        for name, one_kernel in env.forms.items():
+            ar = env.allreduce(n, bits, block, one_kernel)
+            y = env.new_output(x)
+            ar(x, y)
+            env.sync()
+            exact[name] = env.all_true(env.equal(y, want))
+            for _ in range(warmup):
+                ar(x, y)
+            env.sync()
+            env.barrier()
+
+            def calls(ar=ar, y=y):
+                for _ in range(steps):
+                    ar(x, y)
+
+            ms = env.timed(calls)
+            status[name] = int(env.max_over_ranks(float(ar.last_status())))
+            us[name] = env.max_over_ranks(ms / steps * 1e3)
+            ar.close()
+        buf = env.baseline_buffer(x)
+        for _ in range(warmup):
+            env.baseline(buf)
+        env.sync()
+        env.barrier()
+
+        def base_calls():
+            for _ in range(steps):
+                env.baseline(buf)
+
+        ms = env.timed(base_calls)
+        us["nccl_fp16"] = env.max_over_ranks(ms / steps * 1e3)
+        if env.rank == 0:
+            emit({"mode": "collective", "P": P, "bits": bits, "block": block, "elements_per_rank": n,
+                  "bytes_per_rank": 2 * n, "steps": steps, "warmup": warmup,
+                  "us": {k: round(v, 2) for k, v in us.items()},
+                  "wire_bytes_per_rank": wire_bytes_per_rank(P, n, bits, block),
+                  "speedup_vs_nccl_fp16": {k: round(us["nccl_fp16"] / v, 3) for k, v in us.items()
+                                           if k != "nccl_fp16"},
+                  "bit_exact_vs_fused": exact, "wait_status": status,
+                  "timing": env.timing_note})
+
+
+class CudaCollectiveEnv:
+    """The sweep on one GPU per rank: NCCL for the fp16 baseline and the
+    max-over-ranks, a gloo group for the quantized all-reduce's host barriers
+    and handle exchange, inputs drawn on the device (the synthetic recipe's
+    shape: N(0,1) times per-channel log-normal scales over 8192 channels)."""
+
+    timing_note = ("CUDA events on each rank's stream around K calls after W warm-up calls (the host-barrier "
+                   "form's waits included), per call, max over ranks")
+
+    def __init__(self, rank: int, world: int, local: int):
+        import torch
+        import torch.distributed as dist
+
+        import bit_quantized_all_block_b200 as fc
+        from bit_quantized_all_block_b200 import collective
+        self.torch, self.dist, self.fc, self.collective = torch, dist, fc, collective
+        self.rank, self.world = rank, world
+        self.device = torch.device("cuda", local)
+        self.stream = torch.cuda.current_stream()
+        self.host = dist.new_group(backend="gloo", timeout=datetime.timedelta(seconds=120))
+        ids = [None] * world
+        dist.all_gather_object(ids, collective.CudaOps(self.device).device_id(), group=self.host)
+        self.forms = {"host_barrier": False}
+        if world in (2, 4, 8) and not collective.ranks_share_a_device(ids):
+            self.forms["one_kernel"] = True
+
+    def _draw(self, n: int, r: int):
+        torch = self.torch
+        H = 8192 if n % 8192 == 0 else n
+        g = torch.Generator(device=self.device)
+        g.manual_seed(7000 + n)
+        scale = torch.exp(torch.randn(H, device=self.device, generator=g) * 0.5)
+        g.manual_seed(7001 + n + 1000003 * r)
+        return (torch.randn(n // H, H, device=self.device, generator=g) * scale).half().reshape(-1)
+
+    def partial(self, n: int):
+        return self._draw(n, self.rank)
+
+    def expected(self, n: int, bits: int, block: int):
+        xs = [self._draw(n, r) for r in range(self.world)]
+        y = self.fc.fc_quantized_allreduce(xs, bits, block)
+        del xs
+        return y
+
+    def allreduce(self, n, bits, block, one_kernel):
+        return self.collective.QuantizedAllReduce(n, bits, block, group=self.host, one_kernel=one_kernel,
+                                                  timeout=120.0)
+
+    def new_output(self, x):
+        return self.torch.empty_like(x)
+
+    def equal(self, a, b) -> bool:
+        return bool(self.torch.equal(a.view(self.torch.int16), b.view(self.torch.int16)))
+
+    def baseline_buffer(self, x):
+        return x.clone()
+
+    def baseline(self, buf):
+        self.dist.all_reduce(buf)
+
+    def sync(self):
+        self.torch.cuda.synchronize()
+
+    def barrier(self):
+        self.dist.barrier()
+
+    def timed(self, fn) -> float:
+        torch = self.torch
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        a.record(self.stream)
+        fn()
+        b.record(self.stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b)
+
+    def all_true(self, flag: bool) -> bool:
+        t = self.torch.tensor([1 if flag else 0], dtype=self.torch.int32, device=self.device)
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MIN)
+        return bool(t.item())
+
+    def max_over_ranks(self, v: float) -> float:
+        return max_over_ranks(v, self.world)
+
+
+def run_collective(args):
+    """--collective: the sweep under torchrun, one process per GPU (2, 4 or 8
+    for the one-kernel form); one JSON line per point on rank 0."""
+    import torch
+    import torch.distributed as dist
+
+    world, rank, local = dist_setup(args)
+    if world < 2:
+        print(json.dumps({"mode": "collective", "unavailable": "needs 2 or more GPUs, one process per GPU "
+                                                              "(torchrun --nproc-per-node N bench.py --collective)"}),
+              flush=True)
+        return
+    torch.cuda.set_device(local)
+    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+    try:
+        env = CudaCollectiveEnv(rank, world, local)
+        max_bytes = args.collective_max_mb << 20
+        collective_sweep(env, collective_points(world, max_bytes=max_bytes), args.steps, args.warmup,
+                         lambda row: print(json.dumps(row), flush=True))
+        torch.cuda.synchronize()
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -595,6 +797,11 @@ def main():
                     help="decode regime: per-call latency over the 16 KB .. 8 MB per rank message sweep")
     ap.add_argument("--message-sweep", action="store_true",
                     help="the fused all-reduce over 16 KB .. 1 GB per rank (P=4, INT8 and INT4), one line each")
+    ap.add_argument("--collective", action="store_true",
+                    help="under torchrun, one process per GPU: the P-GPU quantized all-reduce (host-barrier and "
+                         "one-kernel forms) against NCCL's fp16 all-reduce over 16 KB .. 1 GB per rank")
+    ap.add_argument("--collective-max-mb", type=int, default=1024,
+                    help="largest message per rank of the --collective sweep (MB)")
     ap.add_argument("--precision-sweep", action="store_true",
                     help="time the fused kernel for every (RS bits, AG bits) in {4,8,16}^2 on the "
                          "workload and report each variant's MSE (one JSON line per variant)")
@@ -613,6 +820,8 @@ def main():
         return run_latency_sweep(args)
     if args.message_sweep:
         return run_message_sweep(args)
+    if args.collective:
+        return run_collective(args)
 
     import torch
     import torch.distributed as dist
@@ -639,6 +848,33 @@ def main():
     s2 = fc.QBuf.empty(w.n, w.bits, w.block)
     stream = torch.cuda.current_stream()
 
+    def staged_once(xs_, y_, s1_, s2_):
+        for r in range(w.P):
+            fc.fc_quantize(xs_[r], w.bits, w.block, out=s1_[r])
+        fc.fc_rs_dequant_sum_requant(s1_, w.bits, w.block, out=s2_)
+        fc.fc_ag_dequant(s2_, tdt, y=y_)
+
+    def staged_timing(xs_, y_, s1_, s2_, small_, flush_):
+        """K staged steps with events between the stages: (mean ms of each of the
+        three stages, total ms of every step)."""
+        marks = []
+        for _ in range(args.steps):
+            if small_:
+                flush_.zero_()
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+            ev[0].record(stream)
+            for r in range(w.P):
+                fc.fc_quantize(xs_[r], w.bits, w.block, out=s1_[r])
+            ev[1].record(stream)
+            fc.fc_rs_dequant_sum_requant(s1_, w.bits, w.block, out=s2_)
+            ev[2].record(stream)
+            fc.fc_ag_dequant(s2_, tdt, y=y_)
+            ev[3].record(stream)
+            marks.append(ev)
+        torch.cuda.synchronize()
+        stage = [sum(m[i].elapsed_time(m[i + 1]) for m in marks) / args.steps for i in range(3)]
+        return stage, [m[0].elapsed_time(m[3]) for m in marks]
+
     variants = args.variant.split(",")
     for vi, variant in enumerate(variants):
         def step(xs_=xs, y_=y):
@@ -647,10 +883,7 @@ def main():
             elif variant == "fused_nopayload":
                 fc.fc_quantized_allreduce(xs_, w.bits, w.block, y=y_)
             else:
-                for r in range(w.P):
-                    fc.fc_quantize(xs_[r], w.bits, w.block, out=s1[r])
-                fc.fc_rs_dequant_sum_requant(s1, w.bits, w.block, out=s2)
-                fc.fc_ag_dequant(s2, tdt, y=y_)
+                staged_once(xs_, y_, s1, s2)
 
         launches_per_step = 1 if variant.startswith("fused") else w.P + 2
 
@@ -666,11 +899,16 @@ def main():
         step_bytes = algorithmic_bytes(w, variant)
         small = step_bytes < L2_FLUSH_THRESHOLD
         graph = None
+        # per-step marks: recorded between the steps (inside the graph as event
+        # record nodes), read after the timed replay for the per-step spread
+        step_marks = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(args.steps + 1)]
         if not small and variant != "staged" and not args.no_graph:
             graph = torch.cuda.CUDAGraph()
             with torch.cuda.graph(graph):
-                for _ in range(args.steps):
+                step_marks[0].record()
+                for i in range(args.steps):
                     step()
+                    step_marks[i + 1].record()
             torch.cuda.synchronize()
             graph.replay()                      # one untimed replay
             torch.cuda.synchronize()
@@ -703,23 +941,7 @@ def main():
             for _ in range(n_ramp):
                 unit()
             if variant == "staged":
-                # events between the stages give each staged kernel its own time
-                marks = []
-                for _ in range(args.steps):
-                    if small:
-                        flush.zero_()
-                    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
-                    ev[0].record(stream)
-                    for r in range(w.P):
-                        fc.fc_quantize(xs[r], w.bits, w.block, out=s1[r])
-                    ev[1].record(stream)
-                    fc.fc_rs_dequant_sum_requant(s1, w.bits, w.block, out=s2)
-                    ev[2].record(stream)
-                    fc.fc_ag_dequant(s2, tdt, y=y)
-                    ev[3].record(stream)
-                    marks.append(ev)
-                torch.cuda.synchronize()
-                stage_ms = [sum(m[i].elapsed_time(m[i + 1]) for m in marks) / args.steps for i in range(3)]
+                stage_ms, step_ms = staged_timing(xs, y, s1, s2, small, flush)
                 ms = sum(stage_ms)
             elif not small:
                 # the K steps are captured once in a CUDA graph and replayed, so
@@ -728,11 +950,14 @@ def main():
                 if graph is not None:
                     graph.replay()
                 else:
-                    for _ in range(args.steps):
+                    step_marks[0].record(stream)
+                    for i in range(args.steps):
                         step()
+                        step_marks[i + 1].record(stream)
                 ev1.record(stream)
                 torch.cuda.synchronize()
                 ms = ev0.elapsed_time(ev1) / args.steps
+                step_ms = [step_marks[i].elapsed_time(step_marks[i + 1]) for i in range(args.steps)]
             else:
                 pairs = []
                 for _ in range(args.steps):
@@ -743,9 +968,20 @@ def main():
                     b.record(stream)
                     pairs.append((a, b))
                 torch.cuda.synchronize()
-                ms = sum(a.elapsed_time(b) for a, b in pairs) / args.steps
+                step_ms = [a.elapsed_time(b) for a, b in pairs]
+                ms = sum(step_ms) / args.steps
+            # the fused line also carries the staged pipeline's roofline, timed in
+            # the same run on the same inputs (its own ramp, K steps)
+            staged_extra = None
+            if variant == "fused":
+                for _ in range(max(1, math.ceil(args.ramp_ms / max(ms * 3, 1e-3)))):
+                    staged_once(xs, y, s1, s2)
+                st_stage_ms, st_step_ms = staged_timing(xs, y, s1, s2, small, flush)
+                staged_extra = (st_stage_ms, st_step_ms)
             barrier()
         ms = max_over_ranks(ms, world)
+        ms_median = max_over_ranks(statistics.median(step_ms), world)
+        ms_min = max_over_ranks(min(step_ms), world)
 
         # ---- end to end through the public API with host buffers -----------------
         # The same calls on the page-locked host inputs and a page-locked host
@@ -849,6 +1085,7 @@ def main():
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
+            "ms_per_step_median": round(ms_median, 5), "ms_per_step_min": round(ms_min, 5),
             "us_per_allreduce": round(ms * 1e3, 2),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f32", "data": "synthetic",
@@ -877,6 +1114,22 @@ def main():
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clocks.summary(),
         }
+
+        if staged_extra is not None:
+            st_stage_ms, st_step_ms = staged_extra
+            st_ms = max_over_ranks(sum(st_stage_ms), world)
+            st_alg = algorithmic_bytes(w, "staged")
+            st_ach = st_alg / (st_ms * 1e-3) / 1e9
+            line["roofline"]["staged"] = {
+                "what": f"the staged pipeline (P k_quantize, k_rs, k_ag launches) on the same inputs, {args.steps} "
+                        f"steps timed after the fused ones",
+                "algorithmic_bytes_per_step": st_alg, "us_per_allreduce": round(st_ms * 1e3, 2),
+                "us_median": round(max_over_ranks(statistics.median(st_step_ms), world) * 1e3, 2),
+                "us_min": round(max_over_ranks(min(st_step_ms), world) * 1e3, 2),
+                "achieved": round(st_ach, 2), "frac": round(st_ach / peak, 4),
+                "kernels_us": {"k_quantize (x P)": round(st_stage_ms[0] * 1e3, 2),
+                               "k_rs": round(st_stage_ms[1] * 1e3, 2), "k_ag": round(st_stage_ms[2] * 1e3, 2)},
+                "gpu_launches": (w.P + 2) * args.steps}
 
         if variant == "staged":
             w2b = payload_bytes(w)

@@ -48,6 +48,15 @@ def test_gpu_arm_line():
     assert rf["bound"] == "hbm" and rf["unit"] == "GB/s" and 0.3 < rf["frac"] < 1.3
     assert abs(rf["frac"] - rf["achieved"] / rf["peak"]) < 1e-3
     assert d["gpu_launches"] == 3                       # one fused launch per timed step
+    # per-step spread beside the mean
+    assert 0 < d["ms_per_step_min"] <= d["ms_per_step_median"]
+    assert d["ms_per_step_min"] <= d["ms_per_step"] * 1.001
+    # the staged pipeline's roofline on the same inputs, in the same line
+    st = rf["staged"]
+    assert st["algorithmic_bytes_per_step"] == 1368391680     # the 70B-shaped INT8 workload, staged
+    assert 0.3 < st["frac"] < 1.3 and abs(st["frac"] - st["achieved"] / rf["peak"]) < 1e-3
+    assert abs(st["us_per_allreduce"] - sum(st["kernels_us"].values())) < 0.05
+    assert st["gpu_launches"] == 3 * (4 + 2)
     assert d["e2e"]["h2d_bytes_per_step"] > 0 and d["e2e"]["d2h_bytes_per_step"] > 0
     assert {"sm_mhz", "sm_max_mhz", "reasons"} <= set(d["clocks"])
     assert d["quality"]["bit_exact_vs_oracle"] is True
