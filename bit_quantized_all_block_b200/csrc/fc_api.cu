@@ -467,27 +467,18 @@ bool make_kmajor_map(CUtensorMap* map, const void* base, bool bf16, uint64_t row
 
 using GemmFnT = cudaError_t (*)(const CUtensorMap&, const CUtensorMap&, const fc::GemmQuantArgs&, cudaStream_t);
 // [dtype][bits == 4][log2(block) - 5]
-const GemmFnT kGemm[2][2][3] = {
-    {{fc::launch_gemm_quant<__half, 8, 32>, fc::launch_gemm_quant<__half, 8, 64>,
-      fc::launch_gemm_quant<__half, 8, 128>},
-     {fc::launch_gemm_quant<__half, 4, 32>, fc::launch_gemm_quant<__half, 4, 64>,
-      fc::launch_gemm_quant<__half, 4, 128>}},
-    {{fc::launch_gemm_quant<__nv_bfloat16, 8, 32>, fc::launch_gemm_quant<__nv_bfloat16, 8, 64>,
-      fc::launch_gemm_quant<__nv_bfloat16, 8, 128>},
-     {fc::launch_gemm_quant<__nv_bfloat16, 4, 32>, fc::launch_gemm_quant<__nv_bfloat16, 4, 64>,
-      fc::launch_gemm_quant<__nv_bfloat16, 4, 128>}},
+#define FC_GEMM_ROW(L, T, B) {L<T, B, 32>, L<T, B, 64>, L<T, B, 128>, L<T, B, 256>}
+const GemmFnT kGemm[2][2][4] = {
+    {FC_GEMM_ROW(fc::launch_gemm_quant, __half, 8), FC_GEMM_ROW(fc::launch_gemm_quant, __half, 4)},
+    {FC_GEMM_ROW(fc::launch_gemm_quant, __nv_bfloat16, 8), FC_GEMM_ROW(fc::launch_gemm_quant, __nv_bfloat16, 4)},
 };
 // The SM-pair kernel (256 x 256 tiles), used when M is a multiple of 256.
-const GemmFnT kGemmPair[2][2][3] = {
-    {{fc::launch_gemm_quant_pair<__half, 8, 32>, fc::launch_gemm_quant_pair<__half, 8, 64>,
-      fc::launch_gemm_quant_pair<__half, 8, 128>},
-     {fc::launch_gemm_quant_pair<__half, 4, 32>, fc::launch_gemm_quant_pair<__half, 4, 64>,
-      fc::launch_gemm_quant_pair<__half, 4, 128>}},
-    {{fc::launch_gemm_quant_pair<__nv_bfloat16, 8, 32>, fc::launch_gemm_quant_pair<__nv_bfloat16, 8, 64>,
-      fc::launch_gemm_quant_pair<__nv_bfloat16, 8, 128>},
-     {fc::launch_gemm_quant_pair<__nv_bfloat16, 4, 32>, fc::launch_gemm_quant_pair<__nv_bfloat16, 4, 64>,
-      fc::launch_gemm_quant_pair<__nv_bfloat16, 4, 128>}},
+const GemmFnT kGemmPair[2][2][4] = {
+    {FC_GEMM_ROW(fc::launch_gemm_quant_pair, __half, 8), FC_GEMM_ROW(fc::launch_gemm_quant_pair, __half, 4)},
+    {FC_GEMM_ROW(fc::launch_gemm_quant_pair, __nv_bfloat16, 8),
+     FC_GEMM_ROW(fc::launch_gemm_quant_pair, __nv_bfloat16, 4)},
 };
+#undef FC_GEMM_ROW
 #ifndef FC_GEMM_PAIR
 #define FC_GEMM_PAIR 1
 #endif
@@ -613,7 +604,7 @@ fc_status fc_gemm_quantize(const void* a, const void* w, fc_dtype dtype, int M, 
                            const fc_qbuf* out, void* partial, int* status, void* stream)
 {
     if ((dtype != FC_FP16 && dtype != FC_BF16) || M <= 0 || N <= 0 || K <= 0 || M % fc::GQ_BM != 0 ||
-        N % fc::GQ_BN != 0 || K % fc::GQ_BK != 0 || (block != 32 && block != 64 && block != 128) ||
+        N % fc::GQ_BN != 0 || K % fc::GQ_BK != 0 || (block != 32 && block != 64 && block != 128 && block != 256) ||
         (out != nullptr && !valid_bits(bits)))
         return FC_ERR_INVALID_ARG;
     if (a == nullptr || w == nullptr || status == nullptr || (out == nullptr && partial == nullptr))
@@ -655,7 +646,7 @@ fc_status fc_gemm_quantize(const void* a, const void* w, fc_dtype dtype, int M, 
     cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), st);
     if (e != cudaSuccess)
         return cuda_fail(e);
-    const int bi = block == 32 ? 0 : block == 64 ? 1 : 2;
+    const int bi = block == 32 ? 0 : block == 64 ? 1 : block == 128 ? 2 : 3;
     e = (pair ? kGemmPair : kGemm)[dtype][qbits == 4][bi](ta, tb, g, st);
     return e == cudaSuccess ? FC_OK : cuda_fail(e);
 }

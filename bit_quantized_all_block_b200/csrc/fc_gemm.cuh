@@ -214,12 +214,80 @@ __device__ __forceinline__ void tile_coords(int tile, int tiles_m, int tiles_n, 
 }
 
 // ---- epilogue: one row's block of `NB` columns ---------------------------------
-// The 16-bit partial values of the block (rounded from fp32, nearest even)
-// are kept as packed pairs; the block is quantized exactly as fc_quantize
-// would quantize the written partial.
+// Blocks of more than 128 columns (256: the tile's whole row) would hold 128
+// registers of packed values, so they take two passes over TMEM instead, 32
+// columns at a time: the first finds the block's extremes of the rounded
+// partial (and writes the partial), the second reads the accumulator again,
+// rounds it the same way and quantizes.  TMEM reads are cheap next to the
+// main loop this epilogue overlaps.
+template <class T, int BITS, int NB>
+__device__ __forceinline__ void epilogue_block_two_pass(uint32_t taddr, const GemmQuantArgs& a, size_t row, int col)
+{
+    using P2 = Pair<T>;
+    using T2 = typename P2::T2;
+    const size_t e = row * (size_t)a.N + col;     // flat element index of the block
+    T2 m = P2::from_f2(make_float2(INFINITY, INFINITY)), M = P2::from_f2(make_float2(-INFINITY, -INFINITY));
+#pragma unroll 1
+    for (int c = 0; c < NB; c += 32) {
+        uint32_t r[32], v16[16];
+        tmem_ld_32cols(taddr + c, r);
+#pragma unroll
+        for (int i = 0; i < 16; i++) {
+            v16[i] = t2_bits(P2::from_f2(make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]))));
+            m = __hmin2(m, as_t2<T2>(v16[i]));
+            M = __hmax2(M, as_t2<T2>(v16[i]));
+        }
+        if (a.partial != nullptr) {
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<T*>(a.partial) + e + c);
+#pragma unroll
+            for (int i = 0; i < 4; i++)
+                st_stream(dst + i, make_uint4(v16[4 * i], v16[4 * i + 1], v16[4 * i + 2], v16[4 * i + 3]));
+        }
+    }
+    if (a.out.codes == nullptr)
+        return;
+    const float mn = fminf(fminf(P2::lo(m), P2::hi(m)), 0.0f);
+    const float mx = fmaxf(fmaxf(P2::lo(M), P2::hi(M)), 0.0f);
+    const BlockQ b = block_q<BITS>(mn, mx);
+    const float cqz = __fsub_rn(b.cq, b.zf);
+    const uint32_t offset = pack_offset<BITS>(b);
+#pragma unroll 1
+    for (int c = 0; c < NB; c += 32) {
+        uint32_t r[32];
+        tmem_ld_32cols(taddr + c, r);
+        uint32_t words[BITS];                     // 32 codes: 8 words at INT8, 4 at INT4
+#pragma unroll
+        for (int g = 0; g < 4; g++) {
+            float q[8];
+#pragma unroll
+            for (int h = 0; h < 4; h++) {
+                const float2 f = P2::to_f2(P2::from_f2(make_float2(__uint_as_float(r[8 * g + 2 * h]),
+                                                                   __uint_as_float(r[8 * g + 2 * h + 1]))));
+                q[2 * h] = fminf(round_product_shifted(f.x, b.inv), cqz);
+                q[2 * h + 1] = fminf(round_product_shifted(f.y, b.inv), cqz);
+            }
+            pack_shifted<BITS>(q, b, offset, words, g);
+        }
+        uint4* cdst = reinterpret_cast<uint4*>(a.out.codes + (e + c) * BITS / 8);
+#pragma unroll
+        for (int i = 0; i < BITS / 4; i++)
+            st_stream(cdst + i, make_uint4(words[4 * i], words[4 * i + 1], words[4 * i + 2], words[4 * i + 3]));
+    }
+    const size_t k = e / NB;
+    a.out.scales[k] = b.s;
+    a.out.zps[k] = zp_byte(b);
+}
+
+// Blocks of up to 128 columns: the 16-bit partial values of the block
+// (rounded from fp32, nearest even) are kept as packed pairs; the block is
+// quantized exactly as fc_quantize would quantize the written partial.
 template <class T, int BITS, int NB>
 __device__ __forceinline__ void epilogue_block(uint32_t taddr, const GemmQuantArgs& a, size_t row, int col)
 {
+    if constexpr (NB > 128) {
+        epilogue_block_two_pass<T, BITS, NB>(taddr, a, row, col);
+        return;
+    }
     using P2 = Pair<T>;
     using T2 = typename P2::T2;
     uint32_t v16[NB / 2];

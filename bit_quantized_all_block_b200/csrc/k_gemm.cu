@@ -1,5 +1,5 @@
 // Launchers and instantiations of the GEMM with the fused step-1 quantizer
-// (fp16/bf16 operands, INT8/INT4 codes, quantization blocks of 32/64/128).
+// (fp16/bf16 operands, INT8/INT4 codes, quantization blocks of 32/64/128/256).
 #include <cuda_runtime.h>
 
 #include <map>
@@ -87,6 +87,10 @@ cudaError_t launch_gemm_quant_pair(const CUtensorMap& ta, const CUtensorMap& tb,
     template cudaError_t launch_gemm_quant<T, 4, 64>(const CUtensorMap&, const CUtensorMap&,      \
                                                      const GemmQuantArgs&, cudaStream_t);         \
     template cudaError_t launch_gemm_quant<T, 4, 128>(const CUtensorMap&, const CUtensorMap&,     \
+                                                      const GemmQuantArgs&, cudaStream_t);        \
+    template cudaError_t launch_gemm_quant<T, 8, 256>(const CUtensorMap&, const CUtensorMap&,     \
+                                                      const GemmQuantArgs&, cudaStream_t);        \
+    template cudaError_t launch_gemm_quant<T, 4, 256>(const CUtensorMap&, const CUtensorMap&,     \
                                                       const GemmQuantArgs&, cudaStream_t);
 FC_GQ(__half)
 FC_GQ(__nv_bfloat16)
@@ -99,6 +103,7 @@ FC_GQ2(__half, 8, 32) FC_GQ2(__half, 8, 64) FC_GQ2(__half, 8, 128)
 FC_GQ2(__half, 4, 32) FC_GQ2(__half, 4, 64) FC_GQ2(__half, 4, 128)
 FC_GQ2(__nv_bfloat16, 8, 32) FC_GQ2(__nv_bfloat16, 8, 64) FC_GQ2(__nv_bfloat16, 8, 128)
 FC_GQ2(__nv_bfloat16, 4, 32) FC_GQ2(__nv_bfloat16, 4, 64) FC_GQ2(__nv_bfloat16, 4, 128)
+FC_GQ2(__half, 8, 256) FC_GQ2(__half, 4, 256) FC_GQ2(__nv_bfloat16, 8, 256) FC_GQ2(__nv_bfloat16, 4, 256)
 #undef FC_GQ2
 
 }  // namespace fc

@@ -172,7 +172,8 @@ fc_status fc_quantized_allreduce_ex(const void* const* x, int P, fc_dtype dtype,
  *           OR-ed with 1 if a pipeline wait inside the kernel gave up (the
  *           kernel then stops early instead of hanging; outputs are invalid).
  * At least one of out / partial must be non-NULL.  Requires M % 128 == 0,
- * N % 256 == 0, K % 64 == 0, block in {32, 64, 128}, bits in {4, 8}; 16-byte
+ * N % 256 == 0, K % 64 == 0, block in {32, 64, 128, 256} (a block lies in one
+ * row of one 256-column output tile), bits in {4, 8}; 16-byte
  * aligned pointers; outputs must not overlap a or w.  Each call runs one
  * persistent kernel (one CTA per SM, 197 KB shared memory, 512 TMEM columns). */
 fc_status fc_gemm_quantize(const void* a, const void* w, fc_dtype dtype, int M, int N, int K, int bits, int block,

@@ -244,7 +244,7 @@ def test_gemm_validation():
                                     if part is not None else None, ctypes.c_void_p(st) if st is not None else None,
                                     None)
 
-    for kw in (dict(M=100), dict(N=100), dict(K=100), dict(M=0), dict(block=256), dict(block=16),
+    for kw in (dict(M=100), dict(N=100), dict(K=100), dict(M=0), dict(block=512), dict(block=16),
                dict(bits=5), dict(dtype=2), dict(out=None, part=None), dict(st=None), dict(a=0)):
         assert call(**kw) == fc.FC_ERR_INVALID_ARG, kw
     assert call(a=a + 8) == fc.FC_ERR_MISALIGNED

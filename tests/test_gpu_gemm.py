@@ -42,7 +42,7 @@ def check_partial(p_gpu, a, w, dtype):
 
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16], ids=["bf16", "fp16"])
 @pytest.mark.parametrize("bits", [8, 4])
-@pytest.mark.parametrize("block", [32, 64, 128])
+@pytest.mark.parametrize("block", [32, 64, 128, 256])
 @pytest.mark.parametrize("M,N,K", [(128, 256, 64), (256, 512, 192), (1024, 1536, 256)])
 def test_gemm_quantize_small(dtype, bits, block, M, N, K):
     a, w = operands(M, N, K, dtype, seed=M + N + K + bits + block)
@@ -99,8 +99,69 @@ def test_tp_pipeline(bits):
 def test_gemm_validation():
     a = torch.zeros(128, 64, dtype=torch.bfloat16, device="cuda")
     w = torch.zeros(256, 64, dtype=torch.bfloat16, device="cuda")
-    for kw in [dict(block=256), dict(bits=3)]:
+    for kw in [dict(block=512), dict(block=16), dict(bits=3)]:
         with pytest.raises(fc.FCError):
             fc.fc_gemm_quantize(a, w, kw.get("bits", 8), kw.get("block", 128))
     with pytest.raises(fc.FCError):
         fc.fc_gemm_quantize(a[:, :32].contiguous(), w[:, :32].contiguous(), 8, 128)   # K % 64
+
+
+def device_operands(M, N, K, dtype, seed):
+    """Seeded operands drawn on the device (the large shapes), with host copies."""
+    g = torch.Generator(device="cuda").manual_seed(seed)
+    a = torch.randn(M, K, device="cuda", generator=g).to(dtype)
+    w = (torch.randn(N, K, device="cuda", generator=g) / K ** 0.5).to(dtype)
+    return a, w
+
+
+def sample_rows(M, seed):
+    """First and last rows, both sides of 128- and 256-row tile edges, random rows."""
+    rng = np.random.default_rng(seed)
+    rows = {0, 1, 127, 128, 255, 256, M // 2 - 1, M // 2, M - 129, M - 128, M - 2, M - 1}
+    rows |= set(int(r) for r in rng.integers(0, M, size=12))
+    return np.array(sorted(r for r in rows if 0 <= r < M))
+
+
+@pytest.mark.parametrize("M,bits,block", [
+    (8192, 8, 128),     # the benchmarked o_proj shape per rank: SM-pair kernel (M % 256 == 0)
+    (8192, 4, 256),     # SM pairs, blocks of a whole tile row
+    (8064, 8, 128),     # M % 256 != 0: the one-SM kernel
+    (8064, 4, 64),
+], ids=["pair-int8-b128", "pair-int4-b256", "onesm-int8-b128", "onesm-int4-b64"])
+def test_gemm_at_the_benchmarked_shape(M, bits, block):
+    """N = 8192, K = 2048 (70B-shaped o_proj slice of one rank of 4): the whole
+    payload equals the oracle's quantization of the GPU's partial; sampled rows
+    of the partial lie within the accumulation bound of the exact product."""
+    N, K, dtype = 8192, 2048, torch.bfloat16
+    a, w = device_operands(M, N, K, dtype, seed=M + bits + block)
+    partial = torch.empty(M, N, dtype=dtype, device="cuda")
+    q, p, status = fc.fc_gemm_quantize(a, w, bits, block, partial=partial)
+    torch.cuda.synchronize()
+    assert int(status[0].item()) == 0
+    rows = sample_rows(M, seed=M)
+    check_partial(p[rows].cpu(), a[rows].cpu(), w.cpu(), dtype)
+    ref = oracle.quantize(p.view(torch.int16).cpu().numpy().view(np.uint16).ravel(), oracle.BF16, bits, block)
+    assert_payload_equal(q, ref, "payload")
+
+
+def test_gemm_down_projection_depth_sampled_rows():
+    """K = 7168 (the down-projection slice): sampled rows of the partial within
+    the accumulation bound, and those rows' codes, scales and zero-points equal
+    the oracle's quantization of the same rows of the GPU partial."""
+    M, N, K, bits, block, dtype = 8192, 8192, 7168, 8, 128, torch.bfloat16
+    a, w = device_operands(M, N, K, dtype, seed=71)
+    partial = torch.empty(M, N, dtype=dtype, device="cuda")
+    q, p, status = fc.fc_gemm_quantize(a, w, bits, block, partial=partial)
+    torch.cuda.synchronize()
+    assert int(status[0].item()) == 0
+    rows = sample_rows(M, seed=7)
+    check_partial(p[rows].cpu(), a[rows].cpu(), w.cpu(), dtype)
+    nb = N // block
+    codes = q.codes.view(M, N).cpu().numpy()
+    scales = q.scales.view(M, nb).cpu().numpy()
+    zps = q.zps.view(M, nb).cpu().numpy()
+    for r in rows:
+        ref = oracle.quantize(p[r].view(torch.int16).cpu().numpy().view(np.uint16), oracle.BF16, bits, block)
+        assert np.array_equal(codes[r], ref.codes), f"row {r}: codes differ"
+        assert np.array_equal(scales[r].view(np.uint32), ref.scales.view(np.uint32)), f"row {r}: scales differ"
+        assert np.array_equal(zps[r], ref.zps), f"row {r}: zero-points differ"
