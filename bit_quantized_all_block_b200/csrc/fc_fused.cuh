@@ -18,7 +18,8 @@
 //    immediate offsets; a thread's 32 bytes of a rank move as one 32-byte
 //    access when the buffers allow it (WIDE), else as two 16-byte ones;
 //  * the P per-rank scale computations of a block are spread over the lanes
-//    of its group (lane r computes rank r) and broadcast with shuffles;
+//    of its group (lane r computes rank r, whose block extremes reach it by a
+//    reduce-scatter over the group's lanes) and broadcast with shuffles;
 //  * the upper code clamp binds only when the block maximum's code rounds to
 //    qmax + 1 -- rare -- so it is checked once per block from the maximum
 //    and applied behind a warp-uniform branch around the per-element minimum
@@ -338,22 +339,68 @@ __global__ void __launch_bounds__(FuShape<P, SMALL>::THREADS, FuShape<P, SMALL>:
 #pragma unroll
             for (int r = 0; r < P; r++)
                 u[r] = local_min_negmax<T, NC>(raw[r]);
-            for (int o = 1; o < Lw; o <<= 1) {
+            // With more than four ranks the lane-split form gathers each lane's
+            // one rank by a reduce-scatter (below); otherwise all-reduce every
+            // rank over the group (at P <= 4 the reduce-scatter's selects cost
+            // more than its saved shuffles: the 70B-shaped INT8 kernel was 2 %
+            // slower with it).
+            constexpr bool scatter = split && P > 4;
+            if constexpr (!scatter) {
+                for (int o = 1; o < Lw; o <<= 1) {
 #pragma unroll
-                for (int r = 0; r < P; r++)
-                    u[r] = t2_bits(__hmin2(as_t2<T2>(u[r]), as_t2<T2>(__shfl_xor_sync(0xffffffffu, u[r], o))));
+                    for (int r = 0; r < P; r++)
+                        u[r] = t2_bits(
+                            __hmin2(as_t2<T2>(u[r]), as_t2<T2>(__shfl_xor_sync(0xffffffffu, u[r], o))));
+                }
             }
             // ---- step-1 scales: one lane per rank when the group is wide enough
             BlockQ mine;
             bool clamp1 = false;
             if constexpr (split) {
-                // lane `me` of the group computes rank me's scale (lanes past
-                // P duplicate rank 0); it needs only that rank's extremes
+                // Lane `me` of the group computes one rank's scale: rank me
+                // (lanes past P: rank 0) after the all-reduce; with the
+                // reduce-scatter, rank (me mod PW), PW = P rounded up to a power
+                // of two (ranks past P stand for rank 0).  The reduce-scatter is
+                // recursive halving over the lane bits below PW: at offset h a
+                // lane keeps the upper half of its remaining ranks if its bit h
+                // is set, else the lower half, and takes the partner's values of
+                // the half it keeps, which leaves lane me with rank (me mod PW)
+                // over the PW lanes that share its higher bits (PW - 1 exchanges
+                // instead of P per round of an all-reduce); the rest of the
+                // group then reduces that one value.
+                constexpr int PW = P <= 1 ? 1 : P <= 2 ? 2 : P <= 4 ? 4 : 8;
                 const int me = lane - grp;
-                const int rr = me < P ? me : 0;
-                uint32_t um;
-                if (L > 32) {                   // blocks that span warps
-                    if (lane == 0) {
+                const int rr = scatter ? ((me & (PW - 1)) < P ? (me & (PW - 1)) : 0) : (me < P ? me : 0);
+                uint32_t um = u[0];
+                if constexpr (scatter) {
+                    uint32_t v[PW];
+#pragma unroll
+                    for (int r = 0; r < PW; r++)
+                        v[r] = u[r < P ? r : 0];
+#pragma unroll
+                    for (int h = PW / 2; h >= 1; h >>= 1) {
+                        const bool up = (lane & h) != 0;
+#pragma unroll
+                        for (int i = 0; i < h; i++) {
+                            const uint32_t keep = up ? v[i + h] : v[i];
+                            const uint32_t send = up ? v[i] : v[i + h];
+                            v[i] = t2_bits(
+                                __hmin2(as_t2<T2>(keep), as_t2<T2>(__shfl_xor_sync(0xffffffffu, send, h))));
+                        }
+                    }
+                    um = v[0];
+                    for (int o = PW; o < Lw; o <<= 1)
+                        um = t2_bits(__hmin2(as_t2<T2>(um), as_t2<T2>(__shfl_xor_sync(0xffffffffu, um, o))));
+                } else if (L <= 32) {
+#pragma unroll
+                    for (int r = 1; r < P; r++)
+                        um = (rr == r) ? u[r] : um;
+                }
+                if (L > 32) {                   // blocks that span warps: the group is the warp
+                    if constexpr (scatter) {
+                        if (me < P)
+                            red16[me][threadIdx.x >> 5] = um;
+                    } else if (lane == 0) {
 #pragma unroll
                         for (int r = 0; r < P; r++)
                             red16[r][threadIdx.x >> 5] = u[r];
@@ -367,11 +414,6 @@ __global__ void __launch_bounds__(FuShape<P, SMALL>::THREADS, FuShape<P, SMALL>:
                     // separates these reads from the next tile's writes.
                     if (B2 == 16)
                         __syncthreads();
-                } else {
-                    um = u[0];
-#pragma unroll
-                    for (int r = 1; r < P; r++)
-                        um = (rr == r) ? u[r] : um;
                 }
                 const T2 t = as_t2<T2>(um);
                 const float mx = fmaxf(-P2::hi(t), 0.0f);
@@ -379,7 +421,8 @@ __global__ void __launch_bounds__(FuShape<P, SMALL>::THREADS, FuShape<P, SMALL>:
                 clamp1 = __any_sync(0xffffffffu, top_code_overflows(mx, mine));
             }
             // (without SPLIT the group is narrower than P lanes, so L < 32 and
-            // every lane holds every rank's extremes in u)
+            // every lane holds every rank's extremes in u; with SPLIT lane r
+            // of the group holds rank r's scale, fetched by shfl_blockq below)
 
             const bool store1 = a.write_step1 && valid;
 #pragma unroll
