@@ -367,18 +367,20 @@ def run_precision_sweep(args, w):
 def run_gemm(args):
     """The GEMM with the fused step-1 quantizer (tensor cores), on the o_proj
     shape of the 70B-shaped workload: one rank's partial of [8192 tokens x 8192
-    hidden] over its K = 8192/4 = 2048 slice, INT8 blocks of 128.  Compared
-    with cuBLAS for the same GEMM followed by the separate quantize kernel."""
+    hidden] over its K = 8192/4 = 2048 slice, INT8 blocks of --gemm-block
+    (default 128).  Compared with cuBLAS for the same GEMM followed by the
+    separate quantize kernel."""
     import torch
 
     import bit_quantized_all_block_b200 as fc
 
     torch.cuda.set_device(0)
     M, N, K = args.gemm_shape
+    B = args.gemm_block
     g = torch.Generator().manual_seed(0)
     a = torch.randn(M, K, generator=g).bfloat16().cuda()
     w = (torch.randn(N, K, generator=g) / K ** 0.5).bfloat16().cuda()
-    q = fc.QBuf.empty(M * N, 8, 128)
+    q = fc.QBuf.empty(M * N, 8, B)
     part = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
     status = torch.zeros(4, dtype=torch.int32, device="cuda")
 
@@ -395,31 +397,31 @@ def run_gemm(args):
         return e0.elapsed_time(e1) / args.steps
 
     with ClockSampler(0) as clocks:
-        ms_fused = timed(lambda: fc.fc_gemm_quantize(a, w, 8, 128, out=q, status=status))
+        ms_fused = timed(lambda: fc.fc_gemm_quantize(a, w, 8, B, out=q, status=status))
     assert int(status[0].item()) == 0, "GEMM pipeline reported a timeout"
-    ms_plain = timed(lambda: fc.fc_gemm_quantize(a, w, 8, 128, partial=part, status=status, quantize=False))
+    ms_plain = timed(lambda: fc.fc_gemm_quantize(a, w, 8, B, partial=part, status=status, quantize=False))
     ms_cublas = timed(lambda: torch.matmul(a, w.t(), out=part))
-    ms_quant = timed(lambda: fc.fc_quantize(part.view(-1), 8, 128, out=q))
+    ms_quant = timed(lambda: fc.fc_quantize(part.view(-1), 8, B, out=q))
     # The whole tensor-parallel layer output for P ranks (the page's setting:
     # each rank's o_proj partial, then the all-reduce), three ways.
     P = args.gemm_ranks
     As = [torch.randn(M, K, generator=g).bfloat16().cuda() for _ in range(P)]
     Ws = [(torch.randn(N, K, generator=g) / K ** 0.5).bfloat16().cuda() for _ in range(P)]
-    q1 = [fc.QBuf.empty(M * N, 8, 128) for _ in range(P)]
-    q2 = fc.QBuf.empty(M * N, 8, 128)
+    q1 = [fc.QBuf.empty(M * N, 8, B) for _ in range(P)]
+    q2 = fc.QBuf.empty(M * N, 8, B)
     parts = [torch.empty(M, N, dtype=torch.bfloat16, device="cuda") for _ in range(P)]
     yb = torch.empty(M * N, dtype=torch.bfloat16, device="cuda")
 
     def layer_fused():
         for r in range(P):
-            fc.fc_gemm_quantize(As[r], Ws[r], 8, 128, out=q1[r], status=status)
-        fc.fc_rs_dequant_sum_requant(q1, 8, 128, out=q2)
+            fc.fc_gemm_quantize(As[r], Ws[r], 8, B, out=q1[r], status=status)
+        fc.fc_rs_dequant_sum_requant(q1, 8, B, out=q2)
         fc.fc_ag_dequant(q2, torch.bfloat16, y=yb)
 
     def layer_unfused(b):
         for r in range(P):
             torch.matmul(As[r], Ws[r].t(), out=parts[r])
-        fc.fc_quantized_allreduce_ex([p_.view(-1) for p_ in parts], b, b, 128, y=yb)
+        fc.fc_quantized_allreduce_ex([p_.view(-1) for p_ in parts], b, b, B, y=yb)
 
     ms_layer_fused = timed(layer_fused)
     ms_layer_cublas_q8 = timed(lambda: layer_unfused(8))
@@ -436,7 +438,7 @@ def run_gemm(args):
         "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
         "us_per_call": round(ms_fused * 1e3, 2), "higher_is_better": True, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": f"o_proj partial per rank M={M} N={N} K={K}, bf16, INT8 block 128"},
+        "config": {"workload": f"o_proj partial per rank M={M} N={N} K={K}, bf16, INT8 block {B}"},
         "roofline": {"bound": "tensor", "achieved": round(tflops, 1), "peak": peak, "unit": "TFLOP/s",
                      "frac": round(tflops / peak, 4), "peak_kind": kind},
         "compare_us": {"fused_gemm_quantize": round(ms_fused * 1e3, 2),
@@ -793,6 +795,7 @@ def main():
                     help="time the tensor-core GEMM with the fused step-1 quantizer (o_proj shape)")
     ap.add_argument("--gemm-shape", type=int, nargs=3, default=[8192, 8192, 2048], metavar=("M", "N", "K"))
     ap.add_argument("--gemm-ranks", type=int, default=4, help="ranks of the tensor-parallel layer comparison")
+    ap.add_argument("--gemm-block", type=int, default=128, help="quantization block of --gemm (32, 64, 128 or 256)")
     ap.add_argument("--latency-sweep", action="store_true",
                     help="decode regime: per-call latency over the 16 KB .. 8 MB per rank message sweep")
     ap.add_argument("--message-sweep", action="store_true",
