@@ -55,6 +55,22 @@ def test_sweep_ragged(dtype, bits, block, P):
 
 @pytest.mark.parametrize("dtype", [oracle.FP16, oracle.BF16], ids=["fp16", "bf16"])
 @pytest.mark.parametrize("bits", [8, 4])
+@pytest.mark.parametrize("block", [32, 64, 128, 1024, 4096])
+@pytest.mark.parametrize("P", [5, 6, 7])
+def test_rank_counts_between_powers_of_two(dtype, bits, block, P):
+    """P = 5..7: the fused kernel gathers each lane's rank extremes by a
+    reduce-scatter over 8 lane slots, three to one of them standing in for
+    rank 0 -- with groups narrower than P (blocks of 32 at E = 16: every lane
+    computes every rank), groups of at least 8 lanes inside a warp (64, 128)
+    and blocks that span warps (1024, 4096); several tiles and a ragged tail."""
+    m = (3 * 4096) // (P * block) + 2
+    n = P * block * m
+    xs = synth.partials(P, n // block, block, dtype, 0.05, 20.0, seed=300 + 10 * P + block + bits + dtype)
+    check_all(xs, dtype, bits, block, staged=(block == 128))
+
+
+@pytest.mark.parametrize("dtype", [oracle.FP16, oracle.BF16], ids=["fp16", "bf16"])
+@pytest.mark.parametrize("bits", [8, 4])
 def test_zeros_and_sparse(dtype, bits):
     P, block = 4, 128
     xs = synth.uniform_partials(P, P * block * 40, dtype, seed=5, zero_frac=0.9)
