@@ -144,3 +144,19 @@ def test_sweep_lines_on_gloo_ranks(world):
         assert row["bit_exact_vs_fused"] == {"host_barrier": True}
         assert row["wait_status"] == {"host_barrier": 0}
         assert row["steps"] == 2 and row["warmup"] == 1 and row["timing"]
+
+
+def test_one_rank_prints_the_unavailable_line():
+    """Without torchrun (one rank) the mode says it needs two or more GPUs and exits 0,
+    before any CUDA call."""
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK")}
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--collective"], capture_output=True,
+                       text=True, cwd=root, env=env, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    (line,) = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    d = json.loads(line)
+    assert d["mode"] == "collective" and "2 or more GPUs" in d["unavailable"]
