@@ -396,12 +396,24 @@ def run_gemm(args):
         torch.cuda.synchronize()
         return e0.elapsed_time(e1) / args.steps
 
+    # The variants are timed in interleaved rounds (each round times every
+    # variant once, K calls each) and each reports its median over the rounds:
+    # under the 1 kW power cap a variant timed later in a process runs slower,
+    # so timing them one after the other would favour whichever goes first.
+    variants = {
+        "fused": lambda: fc.fc_gemm_quantize(a, w, 8, B, out=q, status=status),
+        "plain": lambda: fc.fc_gemm_quantize(a, w, 8, B, partial=part, status=status, quantize=False),
+        "cublas": lambda: torch.matmul(a, w.t(), out=part),
+        "quant": lambda: fc.fc_quantize(part.view(-1), 8, B, out=q),
+    }
+    rounds = {k: [] for k in variants}
     with ClockSampler(0) as clocks:
-        ms_fused = timed(lambda: fc.fc_gemm_quantize(a, w, 8, B, out=q, status=status))
+        for _ in range(5):
+            for k, fn in variants.items():
+                rounds[k].append(timed(fn))
     assert int(status[0].item()) == 0, "GEMM pipeline reported a timeout"
-    ms_plain = timed(lambda: fc.fc_gemm_quantize(a, w, 8, B, partial=part, status=status, quantize=False))
-    ms_cublas = timed(lambda: torch.matmul(a, w.t(), out=part))
-    ms_quant = timed(lambda: fc.fc_quantize(part.view(-1), 8, B, out=q))
+    ms_fused, ms_plain, ms_cublas, ms_quant = (statistics.median(rounds[k]) for k in ("fused", "plain", "cublas",
+                                                                                        "quant"))
     # The whole tensor-parallel layer output for P ranks (the page's setting:
     # each rank's o_proj partial, then the all-reduce), three ways.
     P = args.gemm_ranks
@@ -423,9 +435,12 @@ def run_gemm(args):
             torch.matmul(As[r], Ws[r].t(), out=parts[r])
         fc.fc_quantized_allreduce_ex([p_.view(-1) for p_ in parts], b, b, B, y=yb)
 
-    ms_layer_fused = timed(layer_fused)
-    ms_layer_cublas_q8 = timed(lambda: layer_unfused(8))
-    ms_layer_cublas_16 = timed(lambda: layer_unfused(16))
+    layers = {"fused": layer_fused, "q8": lambda: layer_unfused(8), "u16": lambda: layer_unfused(16)}
+    lr = {k: [] for k in layers}
+    for _ in range(3):
+        for k, fn in layers.items():
+            lr[k].append(timed(fn))
+    ms_layer_fused, ms_layer_cublas_q8, ms_layer_cublas_16 = (statistics.median(lr[k]) for k in ("fused", "q8", "u16"))
     flops = 2.0 * M * N * K
     tflops = flops / (ms_fused * 1e-3) / 1e12
     try:
@@ -441,6 +456,7 @@ def run_gemm(args):
         "config": {"workload": f"o_proj partial per rank M={M} N={N} K={K}, bf16, INT8 block {B}"},
         "roofline": {"bound": "tensor", "achieved": round(tflops, 1), "peak": peak, "unit": "TFLOP/s",
                      "frac": round(tflops / peak, 4), "peak_kind": kind},
+        "timing": "CUDA events around K back-to-back calls; the variants interleaved over 5 rounds, median",
         "compare_us": {"fused_gemm_quantize": round(ms_fused * 1e3, 2),
                        "our_gemm_partial_only": round(ms_plain * 1e3, 2),
                        "cublas_gemm": round(ms_cublas * 1e3, 2), "quantize_kernel": round(ms_quant * 1e3, 2),
