@@ -875,22 +875,44 @@ def main():
 
     def staged_timing(xs_, y_, s1_, s2_, small_, flush_):
         """K staged steps with events between the stages: (mean ms of each of the
-        three stages, total ms of every step)."""
-        marks = []
-        for _ in range(args.steps):
-            if small_:
-                flush_.zero_()
-            ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
-            ev[0].record(stream)
-            for r in range(w.P):
-                fc.fc_quantize(xs_[r], w.bits, w.block, out=s1_[r])
-            ev[1].record(stream)
-            fc.fc_rs_dequant_sum_requant(s1_, w.bits, w.block, out=s2_)
-            ev[2].record(stream)
-            fc.fc_ag_dequant(s2_, tdt, y=y_)
-            ev[3].record(stream)
-            marks.append(ev)
-        torch.cuda.synchronize()
+        three stages, total ms of every step).  Like the fused steps, workloads
+        larger than L2 are timed as one replay of a CUDA graph of the K steps
+        (events recorded between the stages inside the graph), after replays
+        worth --ramp-ms; smaller ones flush L2 before each step, launched one by
+        one."""
+        use_graph = not small_ and not args.no_graph
+        marks = [[torch.cuda.Event(enable_timing=True, external=use_graph) for _ in range(4)]
+                 for _ in range(args.steps)]
+
+        def steps():
+            for ev in marks:
+                if small_:
+                    flush_.zero_()
+                ev[0].record()
+                for r in range(w.P):
+                    fc.fc_quantize(xs_[r], w.bits, w.block, out=s1_[r])
+                ev[1].record()
+                fc.fc_rs_dequant_sum_requant(s1_, w.bits, w.block, out=s2_)
+                ev[2].record()
+                fc.fc_ag_dequant(s2_, tdt, y=y_)
+                ev[3].record()
+
+        if use_graph:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                steps()
+            torch.cuda.synchronize()
+            g.replay()                          # one untimed replay, which also sizes the ramp
+            torch.cuda.synchronize()
+            t_replay = marks[0][0].elapsed_time(marks[-1][3])
+            for _ in range(max(1, math.ceil(args.ramp_ms / max(t_replay, 1e-3)))):
+                g.replay()
+            g.replay()                          # the timed replay: the events hold its times
+            torch.cuda.synchronize()
+            del g
+        else:
+            steps()
+            torch.cuda.synchronize()
         stage = [sum(m[i].elapsed_time(m[i + 1]) for m in marks) / args.steps for i in range(3)]
         return stage, [m[0].elapsed_time(m[3]) for m in marks]
 
@@ -993,8 +1015,9 @@ def main():
             # the same run on the same inputs (its own ramp, K steps)
             staged_extra = None
             if variant == "fused":
-                for _ in range(max(1, math.ceil(args.ramp_ms / max(ms * 3, 1e-3)))):
-                    staged_once(xs, y, s1, s2)
+                if small:       # the graph form carries its own ramp
+                    for _ in range(max(1, math.ceil(args.ramp_ms / max(ms * 3, 1e-3)))):
+                        staged_once(xs, y, s1, s2)
                 st_stage_ms, st_step_ms = staged_timing(xs, y, s1, s2, small, flush)
                 staged_extra = (st_stage_ms, st_step_ms)
             barrier()
@@ -1110,7 +1133,9 @@ def main():
             "dtype": "f32", "data": "synthetic",
             "config": {"workload": w.name, "description": w.describe(), "variant": variant,
                        "parallelism": f"replicas x{world} (P={w.P} ranks emulated per GPU)",
-                       "launch": "CUDA graph of the timed steps" if graph is not None else "stream launches",
+                       "launch": ("CUDA graph of the timed steps"
+                                  if graph is not None or (variant == "staged" and not small and not args.no_graph)
+                                  else "stream launches"),
                        "clock_ramp": (f"{ramp_steps} untimed steps (>= {args.ramp_ms:g} ms) enqueued directly before "
                                       f"the timed region, after the {args.warmup} warm-up steps"),
                        "l2": (f"L2 flushed (512 MB write) before each step, each step timed alone"
@@ -1141,7 +1166,8 @@ def main():
             st_ach = st_alg / (st_ms * 1e-3) / 1e9
             line["roofline"]["staged"] = {
                 "what": f"the staged pipeline (P k_quantize, k_rs, k_ag launches) on the same inputs, {args.steps} "
-                        f"steps timed after the fused ones",
+                        f"steps timed after the fused ones"
+                        + ("" if small else ", one replay of a CUDA graph of them after >= --ramp-ms of replays"),
                 "algorithmic_bytes_per_step": st_alg, "us_per_allreduce": round(st_ms * 1e3, 2),
                 "us_median": round(max_over_ranks(statistics.median(st_step_ms), world) * 1e3, 2),
                 "us_min": round(max_over_ranks(min(st_step_ms), world) * 1e3, 2),
