@@ -1,0 +1,76 @@
+"""PreparedAllReduce: the fused all-reduce with its arguments marshalled once.
+
+CPU: the argument checks happen at construction, before any CUDA call.
+GPU: every call on the same buffers gives the oracle's result for the buffers'
+current contents (inputs rewritten in place between calls), with and without
+payloads, with per-step widths, on a fixed side stream, and equal to the
+regular call."""
+import numpy as np
+import pytest
+import torch
+
+import bit_quantized_all_block_b200 as fc
+import oracle
+from bit_quantized_all_block_b200 import synth
+
+
+def test_arguments_are_checked_at_construction():
+    x = [torch.zeros(4096, dtype=torch.float16) for _ in range(2)]
+    y = torch.zeros(4096, dtype=torch.float16)
+    with pytest.raises(ValueError):
+        fc.PreparedAllReduce([x[0], torch.zeros(2048, dtype=torch.float16)], 8, 8, 128, y=y)
+    with pytest.raises(ValueError):
+        fc.PreparedAllReduce([x[0], torch.zeros(4096, dtype=torch.bfloat16)], 8, 8, 128, y=y)
+    with pytest.raises(ValueError):       # pageable CPU memory is not something a kernel can read
+        fc.PreparedAllReduce(x, 8, 8, 128, y=y)
+    with pytest.raises(TypeError):
+        fc.PreparedAllReduce([torch.zeros(4096, dtype=torch.float32)] * 2, 8, 8, 128, y=y)
+
+
+def _dev(xs_u16, dtype):
+    t = torch.float16 if dtype == oracle.FP16 else torch.bfloat16
+    return [torch.from_numpy(x.view(np.int16).copy()).view(t).cuda() for x in xs_u16]
+
+
+def _host(t):
+    return t.view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("dtype", [oracle.FP16, oracle.BF16], ids=["fp16", "bf16"])
+@pytest.mark.parametrize("bits", [8, 4])
+def test_repeated_calls_follow_the_buffer_contents(dtype, bits):
+    P, block, T, H = 4, 128, 8, 8192          # the decode-shaped message
+    xs = _dev(synth.partials(P, T, H, dtype, 0.0, 1.0, seed=90), dtype)
+    s1 = [fc.QBuf.empty(T * H, bits, block) for _ in range(P)]
+    s2 = fc.QBuf.empty(T * H, bits, block)
+    call = fc.PreparedAllReduce(xs, bits, bits, block, step1=s1, step2=s2)
+    for seed in (91, 92, 93):
+        new = synth.partials(P, T, H, dtype, 0.05, 20.0, seed=seed)
+        for x, h in zip(xs, _dev(new, dtype)):
+            x.copy_(h)                           # same storage, new contents
+        y = call()
+        torch.cuda.synchronize()
+        y_ref, p1, p2 = oracle.allreduce(list(new), dtype, bits, block)
+        assert np.array_equal(_host(y), y_ref), f"seed {seed}: output differs"
+        for q, p in zip(s1 + [s2], p1 + [p2]):
+            assert np.array_equal(q.codes.cpu().numpy(), p.codes)
+            assert np.array_equal(q.scales.cpu().numpy().view(np.uint32), p.scales.view(np.uint32))
+            assert np.array_equal(q.zps.cpu().numpy(), p.zps)
+
+
+@pytest.mark.gpu
+def test_per_step_widths_and_a_side_stream_match_the_regular_call():
+    P, block, T, H, dtype = 8, 256, 16, 4096, oracle.BF16
+    xs = _dev(synth.partials(P, T, H, dtype, 0.001, 50.0, seed=94), dtype)
+    torch.cuda.synchronize()                     # the inputs were written on the default stream
+    side = torch.cuda.Stream()
+    call = fc.PreparedAllReduce(xs, 8, 4, block, stream=side)
+    with torch.cuda.stream(side):
+        y = call()
+    side.synchronize()
+    y_reg = fc.fc_quantized_allreduce_ex(xs, 8, 4, block)
+    torch.cuda.synchronize()
+    assert torch.equal(y.view(torch.int16), y_reg.view(torch.int16))
+    y_ref = oracle.allreduce_ex([_host(x) for x in xs], dtype, 8, 4, block)[0]
+    assert np.array_equal(_host(y), y_ref)
