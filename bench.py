@@ -798,6 +798,8 @@ def main():
     ap.add_argument("--variant", default="fused",
                     help="fused | fused_nopayload | staged, or a comma-separated list (one JSON line each)")
     ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--e2e-chunks", type=int, default=8,
+                    help="token-row chunks of the pipelined host-buffer form of the e2e figure")
     ap.add_argument("--ref-rows", type=int, default=256,
                     help="token rows per rank in one reference (oracle) step")
     ap.add_argument("--cpu-rows", type=int, default=0,
@@ -1047,7 +1049,7 @@ def main():
         # lying in one chunk) on three streams, so the H2D copy of chunk c + 1,
         # the fused call on chunk c and the D2H copy of chunk c - 1 overlap.
         unit = w.H * (w.P * w.block) // math.gcd(w.H, w.P * w.block)
-        nchunks = min(8, w.n // unit) if variant.startswith("fused") else 0
+        nchunks = min(args.e2e_chunks, w.n // unit) if variant.startswith("fused") else 0
         bounds = []
         if nchunks > 1:
             per = (w.n // unit // nchunks) * unit
