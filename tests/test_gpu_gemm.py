@@ -122,17 +122,20 @@ def sample_rows(M, seed):
     return np.array(sorted(r for r in rows if 0 <= r < M))
 
 
-@pytest.mark.parametrize("M,bits,block", [
-    (8192, 8, 128),     # the benchmarked o_proj shape per rank: SM-pair kernel (M % 256 == 0)
-    (8192, 4, 256),     # SM pairs, blocks of a whole tile row
-    (8064, 8, 128),     # M % 256 != 0: the one-SM kernel
-    (8064, 4, 64),
-], ids=["pair-int8-b128", "pair-int4-b256", "onesm-int8-b128", "onesm-int4-b64"])
-def test_gemm_at_the_benchmarked_shape(M, bits, block):
+@pytest.mark.parametrize("M,bits,block,dtype", [
+    (8192, 8, 128, torch.bfloat16),    # the benchmarked o_proj shape per rank: SM-pair kernel (M % 256 == 0)
+    (8192, 4, 256, torch.bfloat16),    # SM pairs, blocks of a whole tile row
+    (8064, 8, 128, torch.bfloat16),    # M % 256 != 0: the one-SM kernel
+    (8064, 4, 64, torch.bfloat16),
+    (8192, 8, 128, torch.float16),     # fp16 operands on both kernels
+    (8064, 4, 256, torch.float16),
+], ids=["pair-int8-b128", "pair-int4-b256", "onesm-int8-b128", "onesm-int4-b64", "pair-fp16-int8-b128",
+        "onesm-fp16-int4-b256"])
+def test_gemm_at_the_benchmarked_shape(M, bits, block, dtype):
     """N = 8192, K = 2048 (70B-shaped o_proj slice of one rank of 4): the whole
     payload equals the oracle's quantization of the GPU's partial; sampled rows
     of the partial lie within the accumulation bound of the exact product."""
-    N, K, dtype = 8192, 2048, torch.bfloat16
+    N, K = 8192, 2048
     a, w = device_operands(M, N, K, dtype, seed=M + bits + block)
     partial = torch.empty(M, N, dtype=dtype, device="cuda")
     q, p, status = fc.fc_gemm_quantize(a, w, bits, block, partial=partial)
@@ -140,7 +143,8 @@ def test_gemm_at_the_benchmarked_shape(M, bits, block):
     assert int(status[0].item()) == 0
     rows = sample_rows(M, seed=M)
     check_partial(p[rows].cpu(), a[rows].cpu(), w.cpu(), dtype)
-    ref = oracle.quantize(p.view(torch.int16).cpu().numpy().view(np.uint16).ravel(), oracle.BF16, bits, block)
+    odt = oracle.BF16 if dtype == torch.bfloat16 else oracle.FP16
+    ref = oracle.quantize(p.view(torch.int16).cpu().numpy().view(np.uint16).ravel(), odt, bits, block)
     assert_payload_equal(q, ref, "payload")
 
 
