@@ -470,54 +470,58 @@ def run_gemm(args):
 
 def run_latency_sweep(args):
     """Decode regime: per-call latency of the fused all-reduce over the message
-    sweep (16 KB .. 8 MB per rank, P=4, INT8 and INT4), measured two ways:
-    back to back inside a CUDA graph (L2 warm: the kernel's own latency) and
-    one call at a time after an L2 flush (cold)."""
+    sweep (16 KB .. 8 MB per rank, P=4, INT8 and INT4), then the decode-shaped
+    message (8 tokens x 8192 hidden) at P=2 (INT8) and P=8 (INT4), measured two
+    ways: back to back inside a CUDA graph (L2 warm: the kernel's own latency)
+    and one call at a time after an L2 flush (cold)."""
     import torch
 
     import bit_quantized_all_block_b200 as fc
 
     torch.cuda.set_device(0)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
-    for bits in (8, 4):
-        for w in synth.message_sweep(bits)[:10]:
-            xs = [torch.from_numpy(x.view(np.int16)).view(torch.float16).cuda() for x in synth.workload_partials(w)]
-            y = torch.empty(w.n, dtype=torch.float16, device="cuda")
-            s1 = [fc.QBuf.empty(w.n, bits, w.block) for _ in range(w.P)]
-            s2 = fc.QBuf.empty(w.n, bits, w.block)
+    extra = [synth.Workload("p2_fp16_8x8192_int8_b128", 2, 8, 8192, synth.FP16, 8, 128, 0.0, 1.0),
+             synth.Workload("p8_fp16_8x8192_int4_b128", 8, 8, 8192, synth.FP16, 4, 128, 0.0, 1.0)]
+    for w in synth.message_sweep(8)[:10] + synth.message_sweep(4)[:10] + extra:
+        bits = w.bits
+        xs = [torch.from_numpy(x.view(np.int16)).view(torch.float16).cuda() for x in synth.workload_partials(w)]
+        y = torch.empty(w.n, dtype=torch.float16, device="cuda")
+        s1 = [fc.QBuf.empty(w.n, bits, w.block) for _ in range(w.P)]
+        s2 = fc.QBuf.empty(w.n, bits, w.block)
 
-            def step():
-                fc.fc_quantized_allreduce(xs, bits, w.block, y=y, step1=s1, step2=s2)
+        def step():
+            fc.fc_quantized_allreduce(xs, bits, w.block, y=y, step1=s1, step2=s2)
 
-            for _ in range(args.warmup):
+        for _ in range(args.warmup):
+            step()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for _ in range(20):
                 step()
-            torch.cuda.synchronize()
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g):
-                for _ in range(20):
-                    step()
-            g.replay()
-            torch.cuda.synchronize()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record()
-            g.replay()
-            e1.record()
-            torch.cuda.synchronize()
-            hot = e0.elapsed_time(e1) * 1e3 / 20
-            pairs = []
-            for _ in range(args.steps):
-                flush.zero_()
-                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                a.record()
-                step()
-                b.record()
-                pairs.append((a, b))
-            torch.cuda.synchronize()
-            cold = sorted(a.elapsed_time(b) * 1e3 for a, b in pairs)[len(pairs) // 2]
-            print(json.dumps({"mode": "latency_sweep", "workload": w.name, "bytes_per_rank": 2 * w.n,
-                              "us_graph_back_to_back": round(hot, 2), "us_cold_l2_median": round(cold, 2),
-                              "input_gbs_back_to_back": round(w.P * w.n * 2 / hot / 1e3, 1)}), flush=True)
-            del g
+        g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        hot = e0.elapsed_time(e1) * 1e3 / 20
+        pairs = []
+        for _ in range(args.steps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            step()
+            b.record()
+            pairs.append((a, b))
+        torch.cuda.synchronize()
+        cold = sorted(a.elapsed_time(b) * 1e3 for a, b in pairs)[len(pairs) // 2]
+        print(json.dumps({"mode": "latency_sweep", "workload": w.name, "P": w.P, "bits": bits,
+                          "bytes_per_rank": 2 * w.n, "us_graph_back_to_back": round(hot, 2),
+                          "us_cold_l2_median": round(cold, 2),
+                          "input_gbs_back_to_back": round(w.P * w.n * 2 / hot / 1e3, 1)}), flush=True)
+        del g
 
 
 def run_message_sweep(args):
