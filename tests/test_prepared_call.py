@@ -74,3 +74,21 @@ def test_per_step_widths_and_a_side_stream_match_the_regular_call():
     assert torch.equal(y.view(torch.int16), y_reg.view(torch.int16))
     y_ref = oracle.allreduce_ex([_host(x) for x in xs], dtype, 8, 4, block)[0]
     assert np.array_equal(_host(y), y_ref)
+
+
+@pytest.mark.gpu
+def test_page_locked_host_buffers():
+    """The prepared call on page-locked host inputs and output (the kernels read
+    and write host memory directly), inputs rewritten in place between calls."""
+    P, block, T, H, dtype = 4, 128, 8, 8192, oracle.FP16
+    xs = [torch.empty(T * H, dtype=torch.float16).pin_memory() for _ in range(P)]
+    y = torch.empty(T * H, dtype=torch.float16).pin_memory()
+    call = fc.PreparedAllReduce(xs, 8, 8, block, y=y)
+    for seed in (95, 96):
+        new = synth.partials(P, T, H, dtype, 0.0, 1.0, seed=seed)
+        for x, h in zip(xs, new):
+            x.copy_(torch.from_numpy(h.view(np.int16).copy()).view(torch.float16))
+        call()
+        torch.cuda.synchronize()
+        y_ref = oracle.allreduce(list(new), dtype, 8, block)[0]
+        assert np.array_equal(y.view(torch.int16).numpy().view(np.uint16), y_ref), f"seed {seed}"
