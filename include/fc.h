@@ -54,7 +54,8 @@
  *     inputs and the output are also 32-byte aligned, the fused all-reduce
  *     (equal widths) and the all-gather step move them with 32-byte accesses,
  *     which is faster; the results are the same bits either way.
- *     Output buffers must not overlap input buffers (checked).
+ *     Output buffers must not overlap input buffers or one another (checked
+ *     before launch: FC_ERR_INVALID_ARG).
  *   - Inputs must be finite.  For bf16, every block whose range is nonzero
  *     must have a range in [2^-100, 2^100]; outside that the scale or its
  *     reciprocal may not be finite and the results are unspecified (the
