@@ -401,7 +401,13 @@ class PreparedAllReduce:
         self._fn = _lib().fc_quantized_allreduce_ex
 
     def __call__(self, stream=None):
-        st = _stream(stream) if stream is not None else (self._stream or _stream(None))
+        # (a fixed stream may be the legacy default stream, handle 0: test for None, not truth)
+        if stream is not None:
+            st = _stream(stream)
+        elif self._stream is not None:
+            st = self._stream
+        else:
+            st = _stream(None)
         status = self._fn(*self._args, st)
         if status != FC_OK:
             raise FCError(status, "fc_quantized_allreduce_ex")

@@ -27,6 +27,59 @@ def test_arguments_are_checked_at_construction():
         fc.PreparedAllReduce([torch.zeros(4096, dtype=torch.float32)] * 2, 8, 8, 128, y=y)
 
 
+class _FakeEntry:
+    """Stands in for the C entry point: records the stream argument of each call."""
+
+    def __init__(self):
+        self.streams = []
+
+    def __call__(self, *args):
+        self.streams.append(args[-1])
+        return fc.FC_OK
+
+
+def _prepared_without_device(fixed):
+    p = fc.PreparedAllReduce.__new__(fc.PreparedAllReduce)
+    p._args, p.y, p._stream, p._fn = (), None, fixed, _FakeEntry()
+    return p
+
+
+class _Stream:
+    def __init__(self, handle):
+        self.cuda_stream = handle
+
+
+def test_a_fixed_stream_with_handle_zero_is_used(monkeypatch):
+    """The legacy default stream has handle 0: fixing it must not fall back to the current stream."""
+    import ctypes
+
+    def no_current_stream(stream):
+        if stream is None:
+            raise AssertionError("the current stream was consulted although a stream was fixed")
+        return ctypes.c_void_p(stream.cuda_stream)
+
+    monkeypatch.setattr(fc, "_stream", no_current_stream)
+    p = _prepared_without_device(ctypes.c_void_p(0))
+    p()
+    p(stream=_Stream(0x1234))                     # a per-call stream still overrides the fixed one
+    assert [s.value for s in p._fn.streams] == [None, 0x1234]
+
+
+def test_without_a_fixed_stream_each_call_takes_the_current_one(monkeypatch):
+    import ctypes
+    seen = []
+
+    def current(stream):
+        seen.append(stream)
+        return ctypes.c_void_p(0x99 if stream is None else stream.cuda_stream)
+
+    monkeypatch.setattr(fc, "_stream", current)
+    p = _prepared_without_device(None)
+    p()
+    p()
+    assert seen == [None, None] and [s.value for s in p._fn.streams] == [0x99, 0x99]
+
+
 def _dev(xs_u16, dtype):
     t = torch.float16 if dtype == oracle.FP16 else torch.bfloat16
     return [torch.from_numpy(x.view(np.int16).copy()).view(t).cuda() for x in xs_u16]
