@@ -210,10 +210,12 @@ __global__ void __launch_bounds__(P2P_THREADS) k_p2p(const __grid_constant__ P2P
         }
         float mn = fminf(acc[0], 0.0f), mx = fmaxf(acc[0], 0.0f);
 #pragma unroll
-        for (int i = 1; i < E; i++) {
-            mn = fminf(mn, acc[i]);
-            mx = fmaxf(mx, acc[i]);
+        for (int i = 1; i + 1 < E; i += 2) {
+            mn = min3(mn, acc[i], acc[i + 1]);
+            mx = max3(mx, acc[i], acc[i + 1]);
         }
+        mn = fminf(mn, acc[E - 1]);
+        mx = fmaxf(mx, acc[E - 1]);
         group_minmax_f32<true>(mn, mx, L, red32);
         const BlockQ b = block_q<BITS>(mn, mx);
         const bool clamp = __any_sync(0xffffffffu, top_code_overflows(mx, b));
@@ -238,16 +240,16 @@ __global__ void __launch_bounds__(P2P_THREADS) k_p2p(const __grid_constant__ P2P
         const size_t k = el >> lg_block;
         uint32_t w[NW];
         load_codes_cg<BITS, NC>(q.codes, el, w);
-        const float s = __ldcg(q.scales + k);
-        const float mz = __uint_as_float(FC_MAGIC_BITS + __ldcg(q.zps + k));
+        const float2 s2 = dup2(__ldcg(q.scales + k));
+        const float2 nmz2 = dup2(-__uint_as_float(FC_MAGIC_BITS + __ldcg(q.zps + k)));
         uint4 ov[NC];
 #pragma unroll
         for (int c = 0; c < NC; c++) {
             float sh[8], v[8];
             chunk_shifted<BITS>(w, c, sh);
 #pragma unroll
-            for (int i = 0; i < 8; i++)
-                v[i] = __fmul_rn(__fsub_rn(sh[i], mz), s);
+            for (int i = 0; i < 8; i += 2)
+                st2(v, i, mul2(add2(ld2(sh, i), nmz2), s2));   // (q - z) * s, the product rounded alone
             ov[c] = narrow8<T>(v);
         }
         store_chunks<NC, false>(y + e, ov);
