@@ -15,7 +15,10 @@ The N > 1 launch (torchrun, one process per GPU) runs an independent replica
 of the whole P-rank problem on every GPU -- the method's ranks are emulated
 inside one GPU, so there is no data-path collective; NCCL carries only the
 barrier and the max-over-ranks of the timings.  ``value`` is the aggregate
-over all GPUs.
+over all GPUs.  After the timed replicas the N > 1 line also carries a
+``collective`` object: the P = N quantized all-reduce across the job's GPUs
+against NCCL's fp16 all-reduce at three message sizes (``--no-collective``
+leaves it out; ``--collective`` runs the full message sweep).
 
 ``--impl reference`` times the CPU oracle (the plain definition the kernels
 are checked against) on a bounded sample of the same workload, on rank 0.
@@ -646,6 +649,14 @@ def collective_sweep(env, points, steps: int, warmup: int, emit, block: int = CO
             ar(x, y)
             env.sync()
             exact[name] = env.all_true(env.equal(y, want))
+            first = int(env.max_over_ranks(float(ar.last_status())))
+            if first != 0:
+                # a bounded wait gave up on some rank: the one-kernel form's
+                # counters no longer match its epochs, so every later call would
+                # give up too (after its wait limit); no rank times this form
+                status[name], us[name] = first, None
+                ar.close()
+                continue
             for _ in range(warmup):
                 ar(x, y)
             env.sync()
@@ -674,10 +685,10 @@ def collective_sweep(env, points, steps: int, warmup: int, emit, block: int = CO
         if env.rank == 0:
             emit({"mode": "collective", "P": P, "bits": bits, "block": block, "elements_per_rank": n,
                   "bytes_per_rank": 2 * n, "steps": steps, "warmup": warmup,
-                  "us": {k: round(v, 2) for k, v in us.items()},
+                  "us": {k: (round(v, 2) if v is not None else None) for k, v in us.items()},
                   "wire_bytes_per_rank": wire_bytes_per_rank(P, n, bits, block),
                   "speedup_vs_nccl_fp16": {k: round(us["nccl_fp16"] / v, 3) for k, v in us.items()
-                                           if k != "nccl_fp16"},
+                                           if k != "nccl_fp16" and v is not None},
                   "bit_exact_vs_fused": exact, "wait_status": status,
                   "timing": env.timing_note})
 
@@ -792,6 +803,32 @@ def run_collective(args):
         dist.destroy_process_group()
 
 
+# Message sizes of the collective object in the N > 1 line: the decode-shaped
+# message (8 x 8192 fp16 per rank) at INT8, the prefill-shaped one
+# (8192 x 8192 fp16 per rank) at INT8 and at INT4, blocks of 128.
+LINE_COLLECTIVE_POINTS = [(8, 8 * 8192), (8, 8192 * 8192), (4, 8192 * 8192)]
+
+
+def collective_in_line(args, world: int, rank: int, local: int):
+    """N > 1: the P = N quantized all-reduce across the job's GPUs (one process
+    per GPU, both forms) against NCCL's fp16 all-reduce at LINE_COLLECTIVE_POINTS,
+    after the timed replicas.  Every rank runs it; rank 0 gets the object for its
+    line.  A failure is reported in the object, not raised."""
+    rows = []
+    try:
+        env = CudaCollectiveEnv(rank, world, local)
+        collective_sweep(env, LINE_COLLECTIVE_POINTS, args.steps, args.warmup, rows.append)
+        err = None
+    except Exception as ex:                         # the replicas' line is printed all the same
+        err = f"{type(ex).__name__}: {ex}"[:300]
+    if rank != 0:
+        return None
+    return {"what": (f"the P = {world} quantized all-reduce across the job's GPUs (one process per GPU; peer "
+                     f"payloads read through IPC mappings) against NCCL's fp16 all-reduce of the same partial, "
+                     f"timed after the replicas"),
+            "points": rows, "error": err}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -827,6 +864,8 @@ def main():
                          "one-kernel forms) against NCCL's fp16 all-reduce over 16 KB .. 1 GB per rank")
     ap.add_argument("--collective-max-mb", type=int, default=1024,
                     help="largest message per rank of the --collective sweep (MB)")
+    ap.add_argument("--no-collective", action="store_true",
+                    help="N > 1: leave the P-GPU collective object out of the default line")
     ap.add_argument("--precision-sweep", action="store_true",
                     help="time the fused kernel for every (RS bits, AG bits) in {4,8,16}^2 on the "
                          "workload and report each variant's MSE (one JSON line per variant)")
@@ -1193,6 +1232,12 @@ def main():
                                    "achieved_gbs": round(b / (t * 1e-3) / 1e9, 1),
                                    "frac": round(b / (t * 1e-3) / 1e9 / peak, 4)}
                                for k, (t, b) in per.items()}
+
+        # ---- N > 1: the method's all-reduce across the job's GPUs (all ranks) ----
+        if world > 1 and vi == 0 and not args.no_collective:
+            coll = collective_in_line(args, world, rank, local)
+            if rank == 0:
+                line["collective"] = coll
 
         # ---- result quality and the CPU baseline (rank 0, N = 1 only) -----------
         if rank == 0:

@@ -245,12 +245,27 @@ def _p2p_tables(P, s1, s2, ctr1, ctr2):
             (ctypes.c_void_p * P)(*[_addr(c) for c in ctr1]), (ctypes.c_void_p * P)(*[_addr(c) for c in ctr2]))
 
 
+class P2PTables:
+    """The payload and counter tables of fc_p2p_allreduce / fc_p2p_allreduce_emulated,
+    marshalled once, for callers that call them many times on the same buffers (the
+    arena of a collective object): building P*P payload descriptors costs tens to
+    hundreds of microseconds of host time, more than a decode-sized call takes on
+    the GPU."""
+
+    def __init__(self, s1, s2, ctr1, ctr2):
+        self.P = len(s2)
+        self.args = _p2p_tables(self.P, s1, s2, ctr1, ctr2)
+
+
 def fc_p2p_allreduce(rank: int, x, y, bits: int, block: int, s1, s2, ctr1, ctr2, epoch: int, status,
-                     ctas_per_rank: int = 0, stream=None):
+                     ctas_per_rank: int = 0, stream=None, tables: P2PTables | None = None):
     """One rank's one-kernel P-GPU all-reduce (see include/fc.h): s1 = P*P payloads (rank p's
-    chunk c at p*P + c), s2 = P owners' payloads, ctr1/ctr2 = P counters (tensors or addresses)."""
-    P = len(s2)
-    a1, a2, c1, c2 = _p2p_tables(P, s1, s2, ctr1, ctr2)
+    chunk c at p*P + c), s2 = P owners' payloads, ctr1/ctr2 = P counters (tensors or addresses);
+    or `tables`, the same four marshalled once (s1, s2, ctr1, ctr2 are then not read)."""
+    if tables is None:
+        tables = P2PTables(s1, s2, ctr1, ctr2)
+    P = tables.P
+    a1, a2, c1, c2 = tables.args
     _check(_lib().fc_p2p_allreduce(rank, P, _dtype_code(x), x.numel(), bits, block,
                                    ctypes.c_void_p(_dev_ptr(x, "x")), ctypes.c_void_p(_dev_ptr(y, "y")),
                                    a1, a2, c1, c2, epoch, ctypes.c_void_p(_addr(status)), ctas_per_rank,
@@ -259,10 +274,14 @@ def fc_p2p_allreduce(rank: int, x, y, bits: int, block: int, s1, s2, ctr1, ctr2,
 
 
 def fc_p2p_allreduce_emulated(xs, ys, bits: int, block: int, s1, s2, ctr1, ctr2, epoch: int, status,
-                              ctas_per_rank: int = 0, stream=None):
+                              ctas_per_rank: int = 0, stream=None, tables: P2PTables | None = None):
     """All P ranks of fc_p2p_allreduce in one cooperative launch on the current GPU."""
     P = len(xs)
-    a1, a2, c1, c2 = _p2p_tables(P, s1, s2, ctr1, ctr2)
+    if tables is None:
+        tables = P2PTables(s1, s2, ctr1, ctr2)
+    if tables.P != P:
+        raise ValueError("the tables are for another number of ranks")
+    a1, a2, c1, c2 = tables.args
     xp = (ctypes.c_void_p * P)(*[_dev_ptr(x, "x") for x in xs])
     yp = (ctypes.c_void_p * P)(*[_dev_ptr(y, "y") for y in ys])
     _check(_lib().fc_p2p_allreduce_emulated(P, _dtype_code(xs[0]), xs[0].numel(), bits, block, xp, yp, a1, a2,

@@ -40,7 +40,7 @@ from __future__ import annotations
 
 from dataclasses import dataclass
 
-from . import (PeerQBuf, fc_ag_dequant, fc_ipc_close, fc_ipc_export, fc_ipc_open, fc_p2p_allreduce,
+from . import (P2PTables, PeerQBuf, fc_ag_dequant, fc_ipc_close, fc_ipc_export, fc_ipc_open, fc_p2p_allreduce,
                fc_payload_sizes, fc_quantize, fc_rs_dequant_sum_requant)
 
 ALIGN = 256
@@ -213,6 +213,13 @@ class QuantizedAllReduce:
             self.status = self.ops.torch.zeros(1, dtype=self.ops.torch.int32, device=self.ops.device)
         self.ops.attach(self.rank, exported)
         self.plan = schedule(self.rank, self.layout)
+        if one_kernel:      # every call passes the same payload and counter addresses: marshal them once
+            L, P = self.layout, self.P
+            self.tables = P2PTables(
+                [self.ops.qbuf(L.step1(p, c), bits, block) for p in range(P) for c in range(P)],
+                [self.ops.qbuf(L.step2(c), bits, block) for c in range(P)],
+                [self.ops.base[p] + L.counters for p in range(P)],
+                [self.ops.base[p] + L.counters + 4 for p in range(P)])
         self.barrier()      # every mapping is in place (and every counter zero) before the first read
 
     def barrier(self):
@@ -239,13 +246,9 @@ class QuantizedAllReduce:
         return y
 
     def _one_kernel_call(self, x, y):
-        L, P = self.layout, self.P
         self.epoch += 1
-        s1 = [self.ops.qbuf(L.step1(p, c), self.bits, self.block) for p in range(P) for c in range(P)]
-        s2 = [self.ops.qbuf(L.step2(c), self.bits, self.block) for c in range(P)]
-        ctr1 = [self.ops.base[p] + L.counters for p in range(P)]
-        ctr2 = [self.ops.base[p] + L.counters + 4 for p in range(P)]
-        fc_p2p_allreduce(self.rank, x, y, self.bits, self.block, s1, s2, ctr1, ctr2, self.epoch, self.status)
+        fc_p2p_allreduce(self.rank, x, y, self.bits, self.block, None, None, None, None, self.epoch, self.status,
+                         tables=self.tables)
         return y
 
     def last_status(self) -> int:

@@ -11,6 +11,7 @@
 #include <cstring>
 #include <map>
 #include <mutex>
+#include <tuple>
 #include <utility>
 
 #include "../../include/fc.h"
@@ -220,32 +221,40 @@ FusedFnT small_variant(fc_dtype dtype, int bits_rs, int bits_ag, int P, int bloc
 
 namespace fc {
 
-cudaError_t persistent_grid(const void* kernel, int threads, size_t n, size_t tile, int* grid)
+cudaError_t kernel_residency(const void* kernel, int threads, int* sms, int* per_sm)
 {
     static std::mutex mu;
-    static std::map<std::pair<int, const void*>, int> cache;  // (device, kernel) -> CTAs
+    // (device, kernel, threads) -> (SMs, co-resident CTAs per SM); the queries
+    // cost microseconds of host time, more than a decode-sized launch
+    static std::map<std::tuple<int, const void*, int>, std::pair<int, int>> cache;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess)
         return e;
-    int ctas = 0;
-    {
-        std::lock_guard<std::mutex> lock(mu);
-        auto it = cache.find({dev, kernel});
-        if (it != cache.end()) {
-            ctas = it->second;
-        } else {
-            int sms = 0, per_sm = 0;
-            e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-            if (e != cudaSuccess)
-                return e;
-            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, 0);
-            if (e != cudaSuccess)
-                return e;
-            ctas = sms * (per_sm > 0 ? per_sm : 1);
-            cache[{dev, kernel}] = ctas;
-        }
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = cache.find({dev, kernel, threads});
+    if (it == cache.end()) {
+        int n_sm = 0, n_cta = 0;
+        e = cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess)
+            return e;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n_cta, kernel, threads, 0);
+        if (e != cudaSuccess)
+            return e;
+        it = cache.emplace(std::make_tuple(dev, kernel, threads), std::make_pair(n_sm, n_cta)).first;
     }
+    *sms = it->second.first;
+    *per_sm = it->second.second;
+    return cudaSuccess;
+}
+
+cudaError_t persistent_grid(const void* kernel, int threads, size_t n, size_t tile, int* grid)
+{
+    int sms = 0, per_sm = 0;
+    cudaError_t e = kernel_residency(kernel, threads, &sms, &per_sm);
+    if (e != cudaSuccess)
+        return e;
+    const int ctas = sms * (per_sm > 0 ? per_sm : 1);
     const size_t tiles = (n + tile - 1) / tile;
     *grid = (int)(tiles < (size_t)ctas ? tiles : (size_t)ctas);
     return cudaSuccess;

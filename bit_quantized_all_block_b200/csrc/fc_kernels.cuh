@@ -75,6 +75,10 @@ inline bool fused_lane_split(int block, int P, bool small)
     return (L < 32 ? L : 32) >= P;
 }
 
+// SMs of the current device and co-resident CTAs of `kernel` per SM at
+// `threads` threads (queried once per device, kernel and thread count).
+cudaError_t kernel_residency(const void* kernel, int threads, int* sms, int* per_sm);
+
 // Persistent grid: enough CTAs of `threads` threads to fill every SM at the
 // kernel's occupancy, never more than there are tiles of `tile` elements.
 cudaError_t persistent_grid(const void* kernel, int threads, size_t n, size_t tile, int* grid);

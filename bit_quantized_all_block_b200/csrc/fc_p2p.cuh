@@ -267,14 +267,9 @@ cudaError_t launch_p2p(const P2PArgs& a, int grid, cudaStream_t st)
 template <class T, int BITS, int P, bool EMU>
 cudaError_t p2p_max_ctas(int* ctas)
 {
-    int dev = 0, sms = 0, per_sm = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e == cudaSuccess)
-        e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (e == cudaSuccess)
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, (const void*)k_p2p<T, BITS, P, EMU>,
-                                                          P2P_THREADS, 0);
-    *ctas = sms * per_sm;
+    int sms = 0, per_sm = 0;
+    const cudaError_t e = kernel_residency((const void*)k_p2p<T, BITS, P, EMU>, P2P_THREADS, &sms, &per_sm);
+    *ctas = sms * per_sm;     // every CTA must be co-resident: no rounding up
     return e;
 }
 

@@ -160,3 +160,96 @@ def test_one_rank_prints_the_unavailable_line():
     (line,) = [l for l in r.stdout.splitlines() if l.startswith("{")]
     d = json.loads(line)
     assert d["mode"] == "collective" and "2 or more GPUs" in d["unavailable"]
+
+
+class _GivesUpOnRank1:
+    """A one-kernel form whose first call reports a bounded wait that gave up, on rank 1 only."""
+
+    def __init__(self, inner, rank, calls):
+        self.inner, self.rank, self.calls = inner, rank, calls
+
+    def __call__(self, x, y):
+        self.calls.append("one_kernel call")
+        return self.inner(x, y)
+
+    def last_status(self):
+        return 1 if self.rank == 1 else 0
+
+    def close(self):
+        self.inner.close()
+
+
+class _EnvWithFailingForm(CpuEnv):
+    def __init__(self, rank, world, dtype):
+        super().__init__(rank, world, dtype)
+        self.forms = {"host_barrier": False, "one_kernel": True}
+
+    def allreduce(self, n, bits, block, one_kernel):
+        inner = super().allreduce(n, bits, block, False)
+        return _GivesUpOnRank1(inner, self.rank, self.calls) if one_kernel else inner
+
+
+def _rank_failing(rank, world, port, points, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        env = _EnvWithFailingForm(rank, world, oracle.FP16)
+        rows = []
+        bench.collective_sweep(env, points, steps=3, warmup=2, emit=rows.append)
+        out[rank] = (rows, env.calls)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_a_form_whose_first_call_gave_up_is_not_timed():
+    """A give-up on any rank is seen by every rank (max over ranks), so no rank times
+    that form: its later calls would give up too, each after the wait limit."""
+    world, n = 2, 2 * 2 * 128 * 2
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    mp.start_processes(_rank_failing, args=(world, _free_port(), [(8, n)], out), nprocs=world,
+                       start_method="spawn")
+    (row,), calls0 = out[0]
+    assert out[1][0] == []
+    for r in range(world):
+        assert out[r][1].count("one_kernel call") == 1      # the checked call only: no warm-up, no timing
+    assert row["wait_status"] == {"host_barrier": 0, "one_kernel": 1}
+    assert row["us"]["one_kernel"] is None and row["us"]["host_barrier"] > 0
+    assert set(row["speedup_vs_nccl_fp16"]) == {"host_barrier"}
+
+
+def _rank_in_line(rank, world, port, fail, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        def make_env(rank_, world_, local):
+            if fail:
+                raise RuntimeError("no peer access")
+            return CpuEnv(rank_, world_, oracle.FP16)
+
+        bench.CudaCollectiveEnv = make_env
+        bench.LINE_COLLECTIVE_POINTS = [(8, world * world * 128), (4, world * world * 128 * 2)]
+
+        class Args:
+            steps, warmup = 2, 1
+
+        out[rank] = bench.collective_in_line(Args, world, rank, 0)
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("fail", [False, True], ids=["runs", "env_fails"])
+def test_collective_object_of_the_multi_gpu_line(fail):
+    world = 2
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    mp.start_processes(_rank_in_line, args=(world, _free_port(), fail, out), nprocs=world, start_method="spawn")
+    assert out[1] is None                                   # rank 0 alone carries it
+    obj = out[0]
+    assert "P = 2" in obj["what"]
+    if fail:
+        assert obj["points"] == [] and "no peer access" in obj["error"]
+    else:
+        assert obj["error"] is None and len(obj["points"]) == 2
+        assert [(p["bits"], p["elements_per_rank"]) for p in obj["points"]] == [(8, 512), (4, 1024)]
+        assert all(p["bit_exact_vs_fused"] == {"host_barrier": True} for p in obj["points"])

@@ -146,3 +146,87 @@ def test_a_rank_that_leaves_ends_the_others_call_with_an_error(stall):
         assert res[1] < (6.0 if stall else 30.0), f"rank {r} waited {res[1]:.1f} s"
     if stall:
         assert any(2.5 < out[r][1] for r in range(world - 1)), "the timeout path was not taken"
+
+
+class _AddressOps:
+    """The one-kernel mode's device side reduced to addresses: each rank's arena
+    sits at a made-up base address (never dereferenced: the kernel call is
+    replaced by a recorder), one made-up device per rank."""
+
+    def __init__(self, rank):
+        import torch
+        self.torch, self.device, self.rank, self.base = torch, torch.device("cpu"), rank, {}
+
+    def alloc(self, nbytes):
+        pass
+
+    def export(self):
+        return 0x10000000 * (self.rank + 1)
+
+    def device_id(self):
+        return f"fake-gpu-{self.rank}"
+
+    def attach(self, rank, exported):
+        self.base = dict(enumerate(exported))
+
+    def qbuf(self, ref, bits, block):
+        from bit_quantized_all_block_b200 import PeerQBuf
+        b = self.base[ref.holder]
+        return PeerQBuf(b + ref.codes, b + ref.scales, b + ref.zps, ref.n, bits, block)
+
+    def new_output(self, x):
+        return x.new_empty(x.shape[0])
+
+    def sync(self):
+        pass
+
+    def close(self):
+        pass
+
+
+def _one_kernel_rank(rank, world, port, n, out):
+    import torch
+
+    from bit_quantized_all_block_b200 import collective
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        calls = []
+
+        def record(rank_, x, y, bits, block, s1, s2, ctr1, ctr2, epoch, status, tables=None):
+            a1, a2, c1, c2 = tables.args
+            calls.append((rank_, epoch, id(tables), [(q.codes, q.scales, q.zps) for q in a1],
+                          [(q.codes, q.scales, q.zps) for q in a2], [c or 0 for c in c1], [c or 0 for c in c2]))
+
+        collective.fc_p2p_allreduce = record
+        ar = collective.QuantizedAllReduce(n, 8, 128, ops=_AddressOps(rank), one_kernel=True, timeout=30.0)
+        x = torch.zeros(n, dtype=torch.float16)
+        for _ in range(3):
+            ar(x)
+        out[rank] = calls
+    finally:
+        dist.destroy_process_group()
+
+
+def test_one_kernel_calls_pass_the_arena_tables_built_once():
+    """Every call hands the kernel the same tables, built at construction: rank p's
+    step-1 payload of chunk c and owner c's step-2 payload at their layout offsets
+    in the holder's arena, the counters at the arena's counter words; the epoch
+    rises by one per call."""
+    world, n = 2, 2 * 128 * 16
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    mp.start_processes(_one_kernel_rank, args=(world, _free_port(), n, out), nprocs=world, start_method="spawn")
+    L = Layout(n, world, 8, 128)
+    base = [0x10000000 * (r + 1) for r in range(world)]
+    want_s1 = [(base[p] + L.step1(p, c).codes, base[p] + L.step1(p, c).scales, base[p] + L.step1(p, c).zps)
+               for p in range(world) for c in range(world)]
+    want_s2 = [(base[c] + L.step2(c).codes, base[c] + L.step2(c).scales, base[c] + L.step2(c).zps)
+               for c in range(world)]
+    for r in range(world):
+        calls = out[r]
+        assert [c[1] for c in calls] == [1, 2, 3] and all(c[0] == r for c in calls)
+        assert len({c[2] for c in calls}) == 1                   # one tables object for every call
+        for _, _, _, s1, s2, c1, c2 in calls:
+            assert s1 == want_s1 and s2 == want_s2
+            assert c1 == [b + L.counters for b in base] and c2 == [b + L.counters + 4 for b in base]

@@ -73,3 +73,33 @@ def test_sweep_on_two_ranks_sharing_one_gpu():
         assert row["wait_status"] == {"host_barrier": 0}
         assert row["us"]["host_barrier"] > 0
         assert row["wire_bytes_per_rank"] == bench.wire_bytes_per_rank(world, n, bits, 128)
+
+
+def _rank_in_line(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    torch.cuda.set_device(0)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=120))
+    try:
+        bench.CudaCollectiveEnv = SharedGpuEnv
+
+        class Args:
+            steps, warmup = 2, 1
+
+        out[rank] = bench.collective_in_line(Args, world, rank, 0)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_collective_object_of_the_multi_gpu_line_at_its_message_sizes():
+    """The N > 1 line's collective object at its own points (the decode-shaped and the
+    prefill-shaped message), both ranks on cuda:0: every point bit-exact."""
+    world = 2
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    mp.start_processes(_rank_in_line, args=(world, _free_port(), out), nprocs=world, start_method="spawn")
+    assert out[1] is None
+    obj = out[0]
+    assert obj["error"] is None, obj["error"]
+    assert [(p["bits"], p["elements_per_rank"]) for p in obj["points"]] == bench.LINE_COLLECTIVE_POINTS
+    for p in obj["points"]:
+        assert p["bit_exact_vs_fused"] == {"host_barrier": True} and p["wait_status"] == {"host_barrier": 0}

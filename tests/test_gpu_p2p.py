@@ -77,6 +77,22 @@ def test_emulated_ranks_match_the_oracle(P, bits, block, dtype, blocks_per_chunk
         _check(R, xs, dtype)
 
 
+@pytest.mark.parametrize("P,bits,block,dtype", [(2, 8, 128, oracle.FP16), (8, 4, 128, oracle.BF16)])
+def test_tables_marshalled_once_serve_every_call(P, bits, block, dtype):
+    """fc.P2PTables built once and passed to every call (the collective object's path):
+    consecutive epochs on new inputs, every output and payload equal to the oracle's."""
+    n = P * block * 9
+    R = Ranks(P, n, dtype, bits, block)
+    tables = fc.P2PTables(R.s1, R.s2, R.ctr1, R.ctr2)
+    for epoch in (1, 2, 3):
+        xs = synth.partials(P, n // block, block, dtype, 0.05, 20.0, seed=90 + epoch + P)
+        fc.fc_p2p_allreduce_emulated(to_dev(xs, dtype), R.ys, bits, block, None, None, None, None, epoch,
+                                     R.status, tables=tables)
+        torch.cuda.synchronize()
+        assert int(R.status.item()) == 0
+        _check(R, xs, dtype)
+
+
 def test_few_ctas_per_rank_loop_over_tiles():
     P, bits, block, dtype = 4, 8, 128, oracle.FP16
     n = P * 128 * 80
