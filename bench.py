@@ -694,10 +694,11 @@ def collective_sweep(env, points, steps: int, warmup: int, emit, block: int = CO
 
 
 class CudaCollectiveEnv:
-    """The sweep on one GPU per rank: NCCL for the fp16 baseline and the
-    max-over-ranks, a gloo group for the quantized all-reduce's host barriers
-    and handle exchange, inputs drawn on the device (the synthetic recipe's
-    shape: N(0,1) times per-channel log-normal scales over 8192 channels)."""
+    """The sweep on one GPU per rank: NCCL for the fp16 baseline, a gloo group
+    for everything else between the ranks (the quantized all-reduce's host
+    barriers and handle exchange, the sweep's barriers, flags and
+    max-over-ranks), inputs drawn on the device (the synthetic recipe's shape:
+    N(0,1) times per-channel log-normal scales over 8192 channels)."""
 
     timing_note = ("CUDA events on each rank's stream around K calls after W warm-up calls (the host-barrier "
                    "form's waits included), per call, max over ranks")
@@ -756,8 +757,13 @@ class CudaCollectiveEnv:
     def sync(self):
         self.torch.cuda.synchronize()
 
+    # Coordination (barriers, flags, timings) runs on the gloo group: if one
+    # rank's call fails, the others' next step ends with a gloo error after the
+    # group's timeout instead of an NCCL operation left waiting, and NCCL runs
+    # only the baseline all-reduce, which every rank reaches past the same gloo
+    # steps.
     def barrier(self):
-        self.dist.barrier()
+        self.dist.barrier(group=self.host)
 
     def timed(self, fn) -> float:
         torch = self.torch
@@ -770,12 +776,14 @@ class CudaCollectiveEnv:
         return a.elapsed_time(b)
 
     def all_true(self, flag: bool) -> bool:
-        t = self.torch.tensor([1 if flag else 0], dtype=self.torch.int32, device=self.device)
-        self.dist.all_reduce(t, op=self.dist.ReduceOp.MIN)
+        t = self.torch.tensor([1 if flag else 0], dtype=self.torch.int32)
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MIN, group=self.host)
         return bool(t.item())
 
     def max_over_ranks(self, v: float) -> float:
-        return max_over_ranks(v, self.world)
+        t = self.torch.tensor([v], dtype=self.torch.float64)
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX, group=self.host)
+        return float(t.item())
 
 
 def run_collective(args):

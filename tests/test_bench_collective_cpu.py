@@ -253,3 +253,43 @@ def test_collective_object_of_the_multi_gpu_line(fail):
         assert obj["error"] is None and len(obj["points"]) == 2
         assert [(p["bits"], p["elements_per_rank"]) for p in obj["points"]] == [(8, 512), (4, 1024)]
         assert all(p["bit_exact_vs_fused"] == {"host_barrier": True} for p in obj["points"])
+
+
+class _FailsOnRank1AtSecondPoint(CpuEnv):
+    def allreduce(self, n, bits, block, one_kernel):
+        if self.rank == 1 and len(self.calls) == 1:
+            raise RuntimeError("peer mapping lost")
+        return super().allreduce(n, bits, block, one_kernel)
+
+
+def _rank_asymmetric(rank, world, port, out):
+    import datetime
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=30))
+    t0 = time.monotonic()
+    try:
+        bench.CudaCollectiveEnv = lambda r, w, local: _FailsOnRank1AtSecondPoint(r, w, oracle.FP16)
+        bench.LINE_COLLECTIVE_POINTS = [(8, world * world * 128), (4, world * world * 128 * 2)]
+
+        class Args:
+            steps, warmup = 2, 1
+
+        obj = bench.collective_in_line(Args, world, rank, 0)
+        out[rank] = (obj, time.monotonic() - t0)
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.timeout(240)
+def test_a_failure_on_one_rank_ends_every_rank_with_an_error_report():
+    """Rank 1 raises inside the sweep, rank 0 does not: rank 1 leaves, rank 0's next
+    step on the gloo group fails instead of waiting for good, and rank 0 still gets
+    its object, with the first point and the error."""
+    world = 2
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    mp.start_processes(_rank_asymmetric, args=(world, _free_port(), out), nprocs=world, start_method="spawn")
+    obj, seconds = out[0]
+    assert out[1][0] is None
+    assert obj["error"] and len(obj["points"]) == 1
+    assert seconds < 120

@@ -3,9 +3,10 @@ drawn on the device, the expected output from the one-GPU fused kernel, the
 real `QuantizedAllReduce` with IPC-mapped arenas, CUDA-event timing) driven by
 `collective_sweep` with two gloo ranks sharing cuda:0.  Only what needs one GPU
 per rank is replaced: NCCL's fp16 all-reduce (here a gloo all-reduce of a host
-copy, a stand-in whose time means nothing) and the NCCL reductions of flags
-and timings (gloo on host tensors).  The one-kernel form is left out by the
-environment itself, since the ranks share a GPU; the host-barrier form may."""
+copy, a stand-in whose time means nothing).  The environment's own barriers,
+flags and max-over-ranks already run on its gloo group.  The one-kernel form is
+left out by the environment itself, since the ranks share a GPU; the
+host-barrier form may."""
 import datetime
 import os
 import socket
@@ -26,16 +27,6 @@ class SharedGpuEnv(bench.CudaCollectiveEnv):
 
     def baseline(self, buf):
         dist.all_reduce(buf)
-
-    def all_true(self, flag):
-        t = torch.tensor([1 if flag else 0], dtype=torch.int32)
-        dist.all_reduce(t, op=dist.ReduceOp.MIN)
-        return bool(t.item())
-
-    def max_over_ranks(self, v):
-        t = torch.tensor([v], dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
 
 
 def _free_port():
