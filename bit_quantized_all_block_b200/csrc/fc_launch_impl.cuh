@@ -5,15 +5,23 @@
 
 namespace fc {
 
+template <class T, int BITS, bool SPAN>
+cudaError_t launch_quantize_as(const QuantArgs& a, cudaStream_t st)
+{
+    int grid = 0;
+    cudaError_t e = persistent_grid((const void*)k_quantize<T, BITS, SPAN>, ST_THREADS, a.n, QuantShape::TILE, &grid);
+    if (e != cudaSuccess)
+        return e;
+    k_quantize<T, BITS, SPAN><<<grid, ST_THREADS, 0, st>>>(a);
+    return cudaGetLastError();
+}
+
 template <class T, int BITS>
 cudaError_t launch_quantize(const QuantArgs& a, cudaStream_t st)
 {
-    int grid = 0;
-    cudaError_t e = persistent_grid((const void*)k_quantize<T, BITS>, ST_THREADS, a.n, QuantShape::TILE, &grid);
-    if (e != cudaSuccess)
-        return e;
-    k_quantize<T, BITS><<<grid, ST_THREADS, 0, st>>>(a);
-    return cudaGetLastError();
+    // blocks wider than a warp's 32 threads reduce through shared memory
+    return a.block > 32 * QuantShape::E ? launch_quantize_as<T, BITS, true>(a, st)
+                                         : launch_quantize_as<T, BITS, false>(a, st);
 }
 
 template <int BITS, int P>

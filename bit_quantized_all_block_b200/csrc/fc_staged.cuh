@@ -3,7 +3,7 @@
 // them (Flash Communication, sciencestack.ai/paper/2412.04964: TL;DR, the
 // quantize -> reduce-scatter -> all-gather structure; Fig. 5 right).
 //
-//   k_quantize<T, BITS>   x_r -> step-1 payload (one rank)
+//   k_quantize<T, BITS, SPAN>   x_r -> step-1 payload (one rank)
 //   k_rs<BITS, P>         P step-1 payloads -> step-2 payload (all chunks)
 //   k_ag<T, BITS>         step-2 payload -> y
 //
@@ -131,8 +131,13 @@ __device__ __forceinline__ void quant_store(const float* v, const BlockQ& b, con
 }
 
 // ---------------------------------------------------------------------------
-// Step 1 on one rank.
-template <class T, int BITS>
+// Step 1 on one rank.  SPAN (blocks that span warps, reduced through shared
+// memory and a CTA barrier; the launcher selects it for blocks above 32*E):
+// the next tile's loads are issued before the block's reduction, so they are
+// in flight during the barrier -- 8 % faster at blocks of 4096.  Within a warp
+// (shuffles only) the loads wait until the scales are known, which measured
+// 1-2 % faster at blocks of 128.
+template <class T, int BITS, bool SPAN>
 __global__ void __launch_bounds__(ST_THREADS) k_quantize(const QuantArgs a)
 {
     using P2 = Pair<T>;
@@ -162,23 +167,37 @@ __global__ void __launch_bounds__(ST_THREADS) k_quantize(const QuantArgs a)
         const size_t e = base + toff;
         const bool valid = e < a.n;
         const size_t k = e >> lg_block;
-        const T2 t = as_t2<T2>(group_min_negmax<T, false>(local_min_negmax<T, NC>(raw), L, red[half]));
-        const float mx = fmaxf(-P2::hi(t), 0.0f);
-        const BlockQ b = block_q<BITS>(fminf(P2::lo(t), 0.0f), mx);
-        const bool clamp = __any_sync(0xffffffffu, top_code_overflows(mx, b));
+        const uint32_t own = local_min_negmax<T, NC>(raw);
         float v[E];
+        BlockQ b;
+        bool clamp;
+        const auto scales = [&] {
+            const T2 t = as_t2<T2>(group_min_negmax<T, false>(own, L, red[half]));
+            const float mx = fmaxf(-P2::hi(t), 0.0f);
+            b = block_q<BITS>(fminf(P2::lo(t), 0.0f), mx);
+            clamp = __any_sync(0xffffffffu, top_code_overflows(mx, b));
+        };
+        const auto widen_and_refill = [&] {
 #pragma unroll
-        for (int c = 0; c < NC; c++) {
-            const uint32_t w[4] = {raw[c].x, raw[c].y, raw[c].z, raw[c].w};
+            for (int c = 0; c < NC; c++) {
+                const uint32_t w[4] = {raw[c].x, raw[c].y, raw[c].z, raw[c].w};
 #pragma unroll
-            for (int h = 0; h < 4; h++) {
-                const float2 f = P2::to_f2(as_t2<T2>(w[h]));
-                v[c * 8 + 2 * h] = f.x;
-                v[c * 8 + 2 * h + 1] = f.y;
+                for (int h = 0; h < 4; h++) {
+                    const float2 f = P2::to_f2(as_t2<T2>(w[h]));
+                    v[c * 8 + 2 * h] = f.x;
+                    v[c * 8 + 2 * h + 1] = f.y;
+                }
             }
+            if (e + stride < a.n)
+                load_chunks<T, NC>(raw, x + e + stride);
+        };
+        if constexpr (SPAN) {
+            widen_and_refill();
+            scales();
+        } else {
+            scales();
+            widen_and_refill();
         }
-        if (e + stride < a.n)
-            load_chunks<T, NC>(raw, x + e + stride);
         if (valid) {
             if (clamp)
                 quant_store<BITS, NC, true>(v, b, a.out, e, j == 0, k);
