@@ -255,6 +255,8 @@ class P2PTables:
     def __init__(self, s1, s2, ctr1, ctr2):
         self.P = len(s2)
         self.args = _p2p_tables(self.P, s1, s2, ctr1, ctr2)
+        # the tables hold raw addresses: keep the tensors behind them allocated
+        self._keep = (list(s1), list(s2), list(ctr1), list(ctr2))
 
 
 def fc_p2p_allreduce(rank: int, x, y, bits: int, block: int, s1, s2, ctr1, ctr2, epoch: int, status,

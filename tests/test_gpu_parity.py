@@ -42,6 +42,21 @@ def test_small_workloads_in_full(w):
 
 @pytest.mark.parametrize("dtype", [oracle.FP16, oracle.BF16], ids=["fp16", "bf16"])
 @pytest.mark.parametrize("bits", [8, 4])
+@pytest.mark.parametrize("block", [2048, 4096])
+@pytest.mark.parametrize("P,m", [(1, 5), (3, 3)])
+def test_blocks_spanning_warps_with_a_partly_empty_last_tile(dtype, bits, block, P, m):
+    """An odd number of blocks of 2048 or 4096: the staged kernels' 8192-element tiles
+    leave the last one partly empty, so some threads of a CTA hold no block but still
+    take part in its cross-warp reduction (the step-1 kernel issues its next loads
+    before that barrier for these blocks)."""
+    n = P * block * m
+    assert (n // block) % 2 == 1
+    xs = synth.partials(P, n // block, block, dtype, 0.05, 20.0, seed=700 + P + bits + dtype + block // 1024)
+    check_all(xs, dtype, bits, block, staged=True)
+
+
+@pytest.mark.parametrize("dtype", [oracle.FP16, oracle.BF16], ids=["fp16", "bf16"])
+@pytest.mark.parametrize("bits", [8, 4])
 @pytest.mark.parametrize("block", BLOCKS)
 @pytest.mark.parametrize("P", [1, 2, 3, 4, 8])
 def test_sweep_ragged(dtype, bits, block, P):

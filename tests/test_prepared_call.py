@@ -145,3 +145,30 @@ def test_page_locked_host_buffers():
         torch.cuda.synchronize()
         y_ref = oracle.allreduce(list(new), dtype, 8, block)[0]
         assert np.array_equal(y.view(torch.int16).numpy().view(np.uint16), y_ref), f"seed {seed}"
+
+
+def test_p2p_tables_keep_their_buffers_alive():
+    """The tables hold raw addresses, so they hold the payload and counter tensors too:
+    dropping the caller's references must not free memory the tables point into."""
+    import gc
+    import weakref
+
+    class Buf:                                  # stands in for a payload with tensors
+        def __init__(self, base):
+            self.base = base
+
+        def struct(self):
+            return fc.fc_qbuf(self.base, self.base + 256, self.base + 512)
+
+    P = 2
+    s1 = [Buf(0x1000 * (i + 1)) for i in range(P * P)]
+    s2 = [Buf(0x9000 * (i + 1)) for i in range(P)]
+    refs = [weakref.ref(b) for b in s1 + s2]
+    tables = fc.P2PTables(s1, s2, [0x100, 0x104], [0x108, 0x10C])
+    del s1, s2
+    gc.collect()
+    assert all(r() is not None for r in refs)
+    assert [q.codes for q in tables.args[0]] == [0x1000 * (i + 1) for i in range(P * P)]
+    del tables
+    gc.collect()
+    assert all(r() is None for r in refs)
