@@ -33,8 +33,9 @@ With one_kernel=True (one GPU per rank) each call is instead a single launch
 of fc_p2p_allreduce: the same three steps inside one cooperative kernel per
 rank, the ranks synchronised by counters in their arenas (system-scope
 atomics and acquire loads through the peer mappings, bounded waits) instead
-of host barriers.  Kernels of different ranks then wait on each other, so
-this mode refuses ranks that share a GPU.
+of host barriers; the kernel's payload and counter tables are built once, at
+construction, since they depend only on the arenas.  Kernels of different
+ranks then wait on each other, so this mode refuses ranks that share a GPU.
 """
 from __future__ import annotations
 
