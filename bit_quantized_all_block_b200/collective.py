@@ -210,7 +210,6 @@ class QuantizedAllReduce:
             dist.all_gather_object(ids, self.ops.device_id(), group=self.host)
             if ranks_share_a_device(ids):
                 raise ValueError("one_kernel needs one GPU per rank: the ranks' kernels wait on each other")
-            self.epoch = 0
             self.status = self.ops.torch.zeros(1, dtype=self.ops.torch.int32, device=self.ops.device)
         self.ops.attach(self.rank, exported)
         self.plan = schedule(self.rank, self.layout)
@@ -247,8 +246,9 @@ class QuantizedAllReduce:
         return y
 
     def _one_kernel_call(self, x, y):
-        self.epoch += 1
-        fc_p2p_allreduce(self.rank, x, y, self.bits, self.block, None, None, None, None, self.epoch, self.status,
+        # epoch 0: the kernel counts its calls on the counters themselves, so a
+        # call captured in a CUDA graph can be replayed
+        fc_p2p_allreduce(self.rank, x, y, self.bits, self.block, None, None, None, None, 0, self.status,
                          tables=self.tables)
         return y
 

@@ -525,7 +525,7 @@ fc_status p2p_common(bool emu, int rank, int P, fc_dtype dtype, size_t n, int bi
 {
     const int pi = P == 2 ? 0 : P == 4 ? 1 : P == 8 ? 2 : -1;
     if (pi < 0 || !valid_bits(bits) || !valid_block(block) || (dtype != FC_FP16 && dtype != FC_BF16) ||
-        n % ((size_t)P * (size_t)block) != 0 || (!emu && (rank < 0 || rank >= P)) || epoch == 0 ||
+        n % ((size_t)P * (size_t)block) != 0 || (!emu && (rank < 0 || rank >= P)) ||
         ctas_per_rank < 0)
         return FC_ERR_INVALID_ARG;
     if (n == 0)

@@ -135,7 +135,14 @@ __global__ void __launch_bounds__(P2P_THREADS) k_p2p(const __grid_constant__ P2P
     const int j = threadIdx.x % L;
     const int lg_block = __ffs(a.block) - 1;
     const size_t toff = (size_t)threadIdx.x * E;
-    const unsigned int target = a.epoch * (unsigned int)a.cpr;
+    // The epoch: given (the k-th call on the counters passes k), or 0 = derived
+    // from this rank's own phase-1 counter.  After k complete calls it holds
+    // k * cpr, and before this CTA counts it can have gained at most cpr - 1
+    // counts of this call, so floor(read / cpr) + 1 is this call's epoch.  No
+    // argument then changes from call to call, so a CUDA graph can replay it.
+    const unsigned int cpr = (unsigned int)a.cpr;
+    const unsigned int epoch = a.epoch != 0 ? a.epoch : __ldcg(a.ctr1[rank]) / cpr + 1;
+    const unsigned int target = epoch * cpr;
 
     // ---- phase 1: quantize every chunk of my partial into S1_rank[c] ----------
     for (size_t base = (size_t)cta * TILE; base < n; base += (size_t)a.cpr * TILE) {

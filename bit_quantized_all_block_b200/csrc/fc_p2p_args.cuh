@@ -23,7 +23,7 @@ struct P2PArgs {
     int block;
     int rank;                         // this rank (ignored by EMU)
     int cpr;                          // CTAs per rank
-    unsigned int epoch;               // 1 for the first call on fresh counters, then 2, 3, ...
+    unsigned int epoch;               // k for the k-th call on the counters, or 0: derived from them
 };
 
 template <class T, int BITS, int P, bool EMU> cudaError_t launch_p2p(const P2PArgs& a, int grid, cudaStream_t st);

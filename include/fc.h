@@ -233,8 +233,13 @@ fc_status fc_ipc_close(void* base);
  *               chunk c (m elements);
  *   ctr1, ctr2  host arrays of P device pointers to rank p's phase counters
  *               (uint32, zero before the first call, never reset);
- *   epoch       1 on the first call with fresh counters, then 2, 3, ...: the
- *               k-th call waits for k * (CTAs per rank) counts;
+ *   epoch       k on the k-th call on these counters (1, 2, 3, ...): the call
+ *               waits for k * (CTAs per rank) counts; or 0: the kernel derives k
+ *               from this rank's phase-1 counter (k-1 complete calls leave
+ *               (k-1) * CTAs on it).  Pass 0 in a call that a CUDA graph
+ *               captures and replays: a replayed explicit epoch is one that
+ *               earlier calls' counts already satisfy, so the ranks would race
+ *               (wrong outputs, no error and no hang);
  *   status      device int of this rank: set to 0 on the stream, OR-ed with 1
  *               when a wait gave up after 2 s (a missing or failed peer); the
  *               outputs are then invalid and the counters no longer agree;
@@ -245,7 +250,8 @@ fc_status fc_ipc_close(void* base);
  * n % (P*block) == 0, 16-byte-aligned payloads, 4-byte-aligned counters.  The
  * buffers the kernel writes or counts on (y, every payload, every counter, the
  * status word) must not overlap one another or x: FC_ERR_INVALID_ARG before
- * launch.  The ranks' calls must use the same n, bits, block, dtype and epoch. */
+ * launch.  The ranks' calls must use the same n, bits, block and dtype, and
+ * the same epoch (or 0 on every rank). */
 fc_status fc_p2p_allreduce(int rank, int P, fc_dtype dtype, size_t n, int bits, int block, const void* x, void* y,
                            const fc_qbuf* s1, const fc_qbuf* s2, unsigned int* const* ctr1,
                            unsigned int* const* ctr2, unsigned int epoch, int* status, int ctas_per_rank,

@@ -138,7 +138,9 @@ def test_p2p_validation():
     assert call(rank=2) == fc.FC_ERR_INVALID_ARG
     assert call(bits=5) == fc.FC_ERR_INVALID_ARG
     assert call(n=4096 + 128) == fc.FC_ERR_INVALID_ARG  # n % (P*block)
-    assert call(epoch=0) == fc.FC_ERR_INVALID_ARG
+    # (epoch 0 is valid: the kernel derives the epoch from the counters.  Every call
+    # here must fail validation, since a call that passed it would launch on these
+    # made-up addresses; epoch 0 is exercised on real buffers in test_gpu_p2p.py)
     assert call(n=0) == fc.FC_OK
     assert lib.fc_p2p_allreduce(0, 2, 0, 4096, 8, 128, x, y, None, s2, ctr, ctr, 1, st, 0, None) == fc.FC_ERR_INVALID_ARG
     assert lib.fc_p2p_allreduce(0, 2, 0, 4096, 8, 128, x, y, s1, s2, ctr, ctr, 1, None, 0, None) == fc.FC_ERR_INVALID_ARG

@@ -212,7 +212,8 @@ def test_one_kernel_calls_pass_the_arena_tables_built_once():
     """Every call hands the kernel the same tables, built at construction: rank p's
     step-1 payload of chunk c and owner c's step-2 payload at their layout offsets
     in the holder's arena, the counters at the arena's counter words; the epoch
-    rises by one per call."""
+    is 0 on every call (the kernel derives it from the counters, so a captured
+    call can be replayed)."""
     world, n = 2, 2 * 128 * 16
     mgr = mp.get_context("spawn").Manager()
     out = mgr.dict()
@@ -225,7 +226,7 @@ def test_one_kernel_calls_pass_the_arena_tables_built_once():
                for c in range(world)]
     for r in range(world):
         calls = out[r]
-        assert [c[1] for c in calls] == [1, 2, 3] and all(c[0] == r for c in calls)
+        assert [c[1] for c in calls] == [0, 0, 0] and all(c[0] == r for c in calls)   # epochs derived on the device
         assert len({c[2] for c in calls}) == 1                   # one tables object for every call
         for _, _, _, s1, s2, c1, c2 in calls:
             assert s1 == want_s1 and s2 == want_s2

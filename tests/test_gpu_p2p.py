@@ -93,6 +93,52 @@ def test_tables_marshalled_once_serve_every_call(P, bits, block, dtype):
         _check(R, xs, dtype)
 
 
+@pytest.mark.parametrize("P,bits,block,dtype", [(2, 8, 128, oracle.FP16), (8, 4, 256, oracle.BF16)])
+def test_epoch_derived_from_the_counters(P, bits, block, dtype):
+    """epoch 0: the kernel derives each call's epoch from its rank's phase-1 counter,
+    also after calls that passed explicit epochs; every call bit-exact with the oracle."""
+    n = P * block * 11
+    R = Ranks(P, n, dtype, bits, block)
+    for epoch, seed in ((1, 60), (0, 61), (0, 62), (4, 63), (0, 64)):
+        xs = synth.partials(P, n // block, block, dtype, 0.05, 20.0, seed=seed + P)
+        assert R.run(to_dev(xs, dtype), epoch) == 0
+        _check(R, xs, dtype)
+
+
+@pytest.mark.parametrize("P,bits,block,dtype", [(4, 8, 128, oracle.FP16), (8, 4, 128, oracle.BF16)])
+def test_call_captured_in_a_cuda_graph_and_replayed(P, bits, block, dtype):
+    """A call with epoch 0 captured once and replayed (the decode-loop pattern): every
+    replay runs the next epoch on the same counters, with the inputs rewritten in
+    place between replays, and gives the oracle's result."""
+    n = P * block * 13
+    R = Ranks(P, n, dtype, bits, block)
+    tables = fc.P2PTables(R.s1, R.s2, R.ctr1, R.ctr2)
+    xs = synth.partials(P, n // block, block, dtype, 0.05, 20.0, seed=70 + P)
+    xd = to_dev(xs, dtype)
+
+    def call():
+        fc.fc_p2p_allreduce_emulated(xd, R.ys, bits, block, None, None, None, None, 0, R.status, tables=tables)
+
+    call()                                   # outside the capture: loads the module, epoch 1
+    torch.cuda.synchronize()
+    assert int(R.status.item()) == 0
+    _check(R, xs, dtype)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        call()
+    for rep in range(3):
+        xs = synth.partials(P, n // block, block, dtype, 0.05, 20.0, seed=80 + rep + P)
+        for d, h in zip(xd, to_dev(xs, dtype)):
+            d.copy_(h)
+        g.replay()
+        torch.cuda.synchronize()
+        assert int(R.status.item()) == 0, f"replay {rep}: a wait gave up"
+        _check(R, xs, dtype)
+    counts = R.ctr.cpu().tolist()        # four complete calls: every counter at 4 x CTAs per rank
+    assert len(set(counts)) == 1 and counts[0] > 0 and counts[0] % 4 == 0, counts
+    del g
+
+
 def test_few_ctas_per_rank_loop_over_tiles():
     P, bits, block, dtype = 4, 8, 128, oracle.FP16
     n = P * 128 * 80
