@@ -263,7 +263,9 @@ def fc_p2p_allreduce(rank: int, x, y, bits: int, block: int, s1, s2, ctr1, ctr2,
                      ctas_per_rank: int = 0, stream=None, tables: P2PTables | None = None):
     """One rank's one-kernel P-GPU all-reduce (see include/fc.h): s1 = P*P payloads (rank p's
     chunk c at p*P + c), s2 = P owners' payloads, ctr1/ctr2 = P counters (tensors or addresses);
-    or `tables`, the same four marshalled once (s1, s2, ctr1, ctr2 are then not read)."""
+    or `tables`, the same four marshalled once (s1, s2, ctr1, ctr2 are then not read).
+    epoch: k for the k-th call on the counters, or 0 to let the kernel derive it (required for
+    a call that a CUDA graph replays)."""
     if tables is None:
         tables = P2PTables(s1, s2, ctr1, ctr2)
     P = tables.P
