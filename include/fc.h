@@ -245,6 +245,12 @@ fc_status fc_ipc_close(void* base);
  *               outputs are then invalid and the counters no longer agree;
  *   ctas_per_rank  0 = as many as can be co-resident (the usual), else a cap;
  *               every rank must use the same value.
+ * The counters count CTAs, and the number of CTAs per rank follows n (a
+ * problem of fewer tiles than fit on the GPU launches one CTA per tile) and
+ * ctas_per_rank: every call on one set of counters must use the same n and
+ * ctas_per_rank, whatever the epoch form (a changed CTA count breaks the
+ * arithmetic of the targets, and the ranks would race).  Use a separate set of
+ * counters for each problem size.
  * The kernel is launched cooperatively (its CTAs wait on each other and on the
  * peers'): no other kernel that waits on this rank may share the GPU.  Requires
  * n % (P*block) == 0, 16-byte-aligned payloads, 4-byte-aligned counters.  The
