@@ -39,6 +39,12 @@ MUTANTS = {
     "zero_block_scale_zero": ("(d == 0.0f) ? 1.0f :", "(d == 0.0f) ? 0.0f :"),
     # the doubly rounded reading: the product rounded to fp32, then to an integer
     "product_rounded_to_fp32_first": ("double t = (double)a * (double)b;", "double t = (double)(float)(a * b);"),
+    "reciprocal_from_range": ("float inv = 1.0f / s;", "float inv = (d == 0.0f) ? 1.0f : (float)qmax / d;"),
+    "extremes_skip_last_element": ("for (int i = 0; i < B; i++) {\n        if (!isfinite(v[i]))",
+                                   "for (int i = 0; i < B - 1; i++) {\n        if (!isfinite(v[i]))"),
+    "dequant_divides_by_reciprocal": ("    return qz * s;", "    return qz / (1.0f / s);"),
+    "sum_drops_last_rank": ("for (int r = 1; r < P; r++) {\n                    float xr",
+                            "for (int r = 1; r < P - 1; r++) {\n                    float xr"),
 }
 
 
