@@ -43,6 +43,10 @@ MUTANTS = {
     "extremes_skip_last_element": ("for (int i = 0; i < B; i++) {\n        if (!isfinite(v[i]))",
                                    "for (int i = 0; i < B - 1; i++) {\n        if (!isfinite(v[i]))"),
     "dequant_divides_by_reciprocal": ("    return qz * s;", "    return qz / (1.0f / s);"),
+    "f16_subnormal_read_as_normal": ("        v = ldexp((double)f, -24);", "        v = ldexp((double)(1024 + f), -25);"),
+    "f16_subnormal_threshold_one_binade_low": ("    if (r < ldexp(1.0, -14))    /* subnormal",
+                                               "    if (r < ldexp(1.0, -15))    /* subnormal"),
+    "f16_largest_finite_overflows": ("    if (r > 65504.0)", "    if (r >= 65504.0)"),
     "sum_drops_last_rank": ("for (int r = 1; r < P; r++) {\n                    float xr",
                             "for (int r = 1; r < P - 1; r++) {\n                    float xr"),
 }
