@@ -293,3 +293,13 @@ def test_a_failure_on_one_rank_ends_every_rank_with_an_error_report():
     assert out[1][0] is None
     assert obj["error"] and len(obj["points"]) == 1
     assert seconds < 120
+
+
+def test_line_points_fit_every_rank_count():
+    """The multi-GPU line's fixed message sizes divide into whole chunks of blocks at
+    every world size of a scaling run (2, 4 and 8 processes).  (Other world sizes get
+    an error in the object: the collective's layout refuses such a message.)"""
+    for P in (2, 4, 8):
+        for bits, n in bench.LINE_COLLECTIVE_POINTS:
+            assert bits in (4, 8)
+            assert n % (P * bench.COLLECTIVE_BLOCK) == 0, (P, n)
